@@ -1,0 +1,256 @@
+"""Plain float64 CPU oracle for scaled dot-product attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY. The tests, the smoke check and the benchmark's CPU
+baseline are the only code that may import this module. The library's
+product path never calls it, and this module shares no code with the CUDA
+kernels.
+
+What it computes is the plain definition from the pages. Each step is a
+small function named after the quantity it produces, so a reader can check it
+against the formula by eye, and the mutation tests can swap one step for a
+known mistake:
+
+  Forward ("Attention Backward Pass (dQ, dK, dV)", section "Forward"):
+      S = Q K^T * scale                 scale = 1/sqrt(d), d = Q.shape[-1]
+      S_ij = -inf for j > i             only if causal (then n == m)
+      P = softmax(S) row by row         stable: subtract the row max
+      O = P V
+  plus the per-row log-sum-exp LSE_i = log sum_j exp(S_ij). The pages do not
+  define it. This oracle reads it as the natural log over the unmasked,
+  already scaled scores, so that P = exp(S - LSE).
+
+  Backward (same page, section "Backward"; "Attention backward" practice set,
+  Problems 2-6):
+      dV = P^T dO
+      dP = dO V^T
+      dS = P * (dP - rowsum(dP * P))    the softmax Jacobian-vector product,
+                                        row by row, no m x m Jacobian
+      dQ = scale * dS K
+      dK = scale * dS^T Q
+  P is recomputed from Q and K inside the backward pass, as that page's
+  "Edge cases and conventions" asks. The row sum is taken over dP * P exactly
+  as printed, not through the rowsum(dO * O) identity, so the identity stays
+  an independent check.
+
+Evaluation order. Each query row is independent in the forward pass and in
+dS, and dK and dV are sums over query rows. The head-level functions
+therefore apply the definition to ``row_block`` query rows at a time, so that
+the n x m score matrix of a long sequence never has to exist at once.
+Within a block nothing is fused or reordered.
+
+Pins (tests/test_oracle.py): the worked examples of "Attention Backward Pass
+(dQ, dK, dV)" (section "Examples"); the loss value printed in "Lesson 4 - The
+Backward Pass for Attention" (section "A Scalar Loss So dout Is Known"),
+reproduced from the same seed; central finite differences of
+L = sum(O * dO); float64 torch autograd of the library's
+scaled_dot_product_attention; the explicit softmax Jacobian diag(a) - a a^T
+("Lesson 4", Exercise 2); the rowsum(dP * P) = rowsum(dO * O) identity
+("Attention Backpropagation: Step by step derivation", "Gradient of S");
+exact zeros at masked positions ("Attention backward", Problem 8); and
+mutation tests that plant each of the pages' wrong variants and check that
+the pins catch it. No function here is left unpinned.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "default_scale", "scores", "apply_causal_mask", "row_softmax",
+    "grad_v", "grad_p", "softmax_jvp", "grad_q", "grad_k",
+    "head_forward", "head_backward", "head_backward_sampled",
+    "attention_forward", "attention_backward",
+]
+
+ROW_BLOCK = 256
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) with d the width of Q and K ("Forward": d = Q.shape[-1])."""
+    return 1.0 / math.sqrt(d)
+
+
+# --------------------------------------------------------------------------
+# Forward steps
+# --------------------------------------------------------------------------
+def scores(Qb: np.ndarray, K: np.ndarray, scale: float) -> np.ndarray:
+    """S = Q K^T * scale for a block of query rows ("Forward"; Problem 1)."""
+    return (Qb @ K.T) * scale
+
+
+def apply_causal_mask(S: np.ndarray, row0: int) -> np.ndarray:
+    """Set S_ij = -inf where key j lies after query i, before the softmax.
+
+    ``row0`` is the global index of the block's first query row. The
+    diagonal is kept ("Attention backward", Problem 8: the mask keeps the
+    diagonal and everything below it).
+    """
+    rows = np.arange(row0, row0 + S.shape[0])[:, None]
+    cols = np.arange(S.shape[1])[None, :]
+    return np.where(cols > rows, -np.inf, S)
+
+
+def row_softmax(S: np.ndarray):
+    """Row-wise softmax with the row max subtracted, and the row LSE.
+
+    Returns (P, lse) with P = exp(S - lse) and lse = max + log(sum exp(S - max)).
+    Masked entries (-inf) give exactly 0 in P.
+    """
+    mx = S.max(axis=-1, keepdims=True)
+    e = np.exp(S - mx)
+    total = e.sum(axis=-1, keepdims=True)
+    P = e / total
+    lse = (mx + np.log(total))[:, 0]
+    return P, lse
+
+
+# --------------------------------------------------------------------------
+# Backward steps
+# --------------------------------------------------------------------------
+def grad_v(P: np.ndarray, dO: np.ndarray) -> np.ndarray:
+    """dV = P^T dO ("Backward"; Problem 2)."""
+    return P.T @ dO
+
+
+def grad_p(dO: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """dP = dO V^T ("Backward"; Problem 3)."""
+    return dO @ V.T
+
+
+def softmax_jvp(P: np.ndarray, dP: np.ndarray) -> np.ndarray:
+    """dS = P * (dP - rowsum(dP * P)), row by row ("Backward"; Problem 4)."""
+    return P * (dP - (dP * P).sum(axis=-1, keepdims=True))
+
+
+def grad_q(dS: np.ndarray, K: np.ndarray, scale: float) -> np.ndarray:
+    """dQ = scale * dS K ("Backward"; Problem 5)."""
+    return scale * (dS @ K)
+
+
+def grad_k(dS: np.ndarray, Q: np.ndarray, scale: float) -> np.ndarray:
+    """dK = scale * dS^T Q ("Backward"; Problem 6)."""
+    return scale * (dS.T @ Q)
+
+
+# --------------------------------------------------------------------------
+# One head: Q (n,d), K (m,d), V (m,dv), dO (n,dv)
+# --------------------------------------------------------------------------
+def _check_head(Q, K, V, causal):
+    n, d = Q.shape
+    m, dk = K.shape
+    if dk != d or V.shape[0] != m:
+        raise ValueError(f"shape mismatch Q{Q.shape} K{K.shape} V{V.shape}")
+    if causal and n != m:
+        raise ValueError("causal attention needs as many queries as keys")
+
+
+def _block_probs(Q, K, r0, r1, causal, scale):
+    S = scores(Q[r0:r1], K, scale)
+    if causal:
+        S = apply_causal_mask(S, r0)
+    return row_softmax(S)
+
+
+def head_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK):
+    """Return (O, lse) for one head, in float64."""
+    Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
+    _check_head(Q, K, V, causal)
+    scale = default_scale(Q.shape[1]) if scale is None else float(scale)
+    n = Q.shape[0]
+    O = np.empty((n, V.shape[1]))
+    lse = np.empty(n)
+    for r0 in range(0, n, row_block):
+        r1 = min(n, r0 + row_block)
+        P, lse[r0:r1] = _block_probs(Q, K, r0, r1, causal, scale)
+        O[r0:r1] = P @ V
+    return O, lse
+
+
+def head_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
+    """Return (dQ, dK, dV) for one head, in float64, recomputing P."""
+    Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, dO))
+    _check_head(Q, K, V, causal)
+    scale = default_scale(Q.shape[1]) if scale is None else float(scale)
+    n = Q.shape[0]
+    dQ = np.empty_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for r0 in range(0, n, row_block):
+        r1 = min(n, r0 + row_block)
+        P, _ = _block_probs(Q, K, r0, r1, causal, scale)
+        dV += grad_v(P, dO[r0:r1])
+        dP = grad_p(dO[r0:r1], V)
+        dS = softmax_jvp(P, dP)
+        dQ[r0:r1] = grad_q(dS, K, scale)
+        dK += grad_k(dS, Q[r0:r1], scale)
+    return dQ, dK, dV
+
+
+def head_backward_sampled(Q, K, V, dO, q_rows, k_rows, causal=False,
+                          scale=None, row_block=ROW_BLOCK):
+    """Selected rows of O, lse, dQ (query rows) and of dK, dV (key rows).
+
+    The same steps as head_forward/head_backward. dQ row i needs only query
+    row i's block; dK and dV rows j need column j of P and dS over every
+    query row, so every block is still visited, but only the selected
+    columns enter the two key-side products.
+    """
+    Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, dO))
+    _check_head(Q, K, V, causal)
+    scale = default_scale(Q.shape[1]) if scale is None else float(scale)
+    q_rows = np.asarray(q_rows, dtype=np.int64)
+    k_rows = np.asarray(k_rows, dtype=np.int64)
+    n = Q.shape[0]
+    O_s = np.empty((len(q_rows), V.shape[1]))
+    lse_s = np.empty(len(q_rows))
+    dQ_s = np.empty((len(q_rows), Q.shape[1]))
+    dK_s = np.zeros((len(k_rows), K.shape[1]))
+    dV_s = np.zeros((len(k_rows), V.shape[1]))
+    for r0 in range(0, n, row_block):
+        r1 = min(n, r0 + row_block)
+        P, lse = _block_probs(Q, K, r0, r1, causal, scale)
+        dP = grad_p(dO[r0:r1], V)
+        dS = softmax_jvp(P, dP)
+        dV_s += grad_v(P[:, k_rows], dO[r0:r1])
+        dK_s += grad_k(dS[:, k_rows], Q[r0:r1], scale)
+        sel = np.nonzero((q_rows >= r0) & (q_rows < r1))[0]
+        if len(sel):
+            loc = q_rows[sel] - r0
+            O_s[sel] = P[loc] @ V
+            lse_s[sel] = lse[loc]
+            dQ_s[sel] = grad_q(dS[loc], K, scale)
+    return O_s, lse_s, dQ_s, dK_s, dV_s
+
+
+# --------------------------------------------------------------------------
+# Batched [..., N, d] front ends, mirroring the pages' two calls
+# --------------------------------------------------------------------------
+def _heads(*arrays):
+    lead = arrays[0].shape[:-2]
+    flat = [np.asarray(a, dtype=np.float64).reshape((-1,) + a.shape[-2:])
+            for a in arrays]
+    return lead, flat
+
+
+def attention_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK):
+    """O and LSE for tensors shaped [..., n, d]; scale defaults to 1/sqrt(d)."""
+    lead, (q, k, v) = _heads(Q, K, V)
+    O = np.empty(q.shape[:2] + (v.shape[2],))
+    lse = np.empty(q.shape[:2])
+    for h in range(q.shape[0]):
+        O[h], lse[h] = head_forward(q[h], k[h], v[h], causal, scale, row_block)
+    return O.reshape(lead + O.shape[1:]), lse.reshape(lead + lse.shape[1:])
+
+
+def attention_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
+    """(dQ, dK, dV) with the shapes of Q, K, V, for tensors shaped [..., N, d]."""
+    lead, (q, k, v, do) = _heads(Q, K, V, dO)
+    dQ = np.empty_like(q)
+    dK = np.empty_like(k)
+    dV = np.empty_like(v)
+    for h in range(q.shape[0]):
+        dQ[h], dK[h], dV[h] = head_backward(q[h], k[h], v[h], do[h], causal,
+                                            scale, row_block)
+    return (dQ.reshape(lead + dQ.shape[1:]), dK.reshape(lead + dK.shape[1:]),
+            dV.reshape(lead + dV.shape[1:]))
