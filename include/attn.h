@@ -1,0 +1,143 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) scaled dot-product attention library.
+ *
+ * The library computes the forward pass of scaled dot-product attention, which
+ * saves one log-sum-exp per query row, and the backward pass, which turns the
+ * upstream gradient dO into dQ, dK and dV:
+ *
+ *   forward   S = scale * Q K^T,  S_ij = -inf for j > i if causal,
+ *             P = softmax(S) row by row,  O = P V,  LSE_i = log sum_j exp(S_ij)
+ *   backward  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+ *             dQ = scale * dS K,  dK = scale * dS^T Q
+ *
+ * Sources: "Attention Backward Pass (dQ, dK, dV) - Transformer Architecture",
+ * sections "Forward", "Backward" and "Expected Return Format" (the two calls,
+ * the shapes, the causal rule n == m); "Attention backward" (eulerpad practice
+ * set), Problems 2-6 and 8 (each gradient, the exact zeros under the mask);
+ * "Attention Backpropagation: Step by step derivation", section "Gradient of S"
+ * (rowsum(dP * P) = rowsum(dO * O), which lets the backward pass use O instead
+ * of a row of P). The LSE output is not on the pages: it is the natural log of
+ * the row's softmax denominator over the unmasked, already scaled scores, so
+ * that the backward pass can rebuild P = exp(S - LSE) without storing P.
+ *
+ * Conventions shared by every call
+ *  - Tensors are dense, row-major [B, H, N, width] arrays in device memory,
+ *    owned by the caller. The library never allocates device memory and never
+ *    frees a caller's pointer.
+ *  - Every pointer must be 16-byte aligned. LSE is [B, H, n] fp32.
+ *  - Q, K, V, O, dO, dQ, dK, dV share one element type, attn_dtype_t. LSE and
+ *    the backward workspace are fp32 whatever the element type.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and never synchronise the host.
+ *  - Every argument is checked before anything is launched. A status other
+ *    than ATTN_OK means that nothing was launched and no output was written.
+ *    ATTN_ERR_CUDA reports a launch error from the CUDA runtime.
+ *  - Kernel paths: bf16 with d == dv in {64, 128} runs on the tcgen05 tensor
+ *    cores (TMA-fed, TMEM accumulators). f32, and bf16 of any other width up
+ *    to 128, runs on a CUDA-core (FFMA) path in fp32 arithmetic.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_NULL = 1,           /* a required pointer is NULL                     */
+    ATTN_ERR_SHAPE = 2,          /* a size is < 1, causal with n != m, or too big  */
+    ATTN_ERR_DTYPE = 3,          /* unknown attn_dtype_t                           */
+    ATTN_ERR_UNSUPPORTED = 4,    /* valid request this build does not implement    */
+    ATTN_ERR_ALIGN = 5,          /* a pointer is not 16-byte aligned               */
+    ATTN_ERR_WORKSPACE = 6,      /* workspace NULL or smaller than required        */
+    ATTN_ERR_CUDA = 7,           /* the CUDA runtime reported an error             */
+    ATTN_ERR_DEVICE_TIMEOUT = 8  /* a kernel gave up a bounded wait (see below)    */
+} attn_status_t;
+
+typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype_t;
+
+/* Which kernels a call may use. ATTN_PATH_AUTO picks the tensor-core path
+ * where it applies (bf16, d == dv in {64, 128}) and the CUDA-core path
+ * otherwise. ATTN_PATH_SIMT forces the CUDA-core path. ATTN_PATH_TENSOR
+ * requires the tensor-core path and makes other shapes ATTN_ERR_UNSUPPORTED.
+ * The setting is process-wide and applies to calls made after it. */
+typedef enum { ATTN_PATH_AUTO = 0, ATTN_PATH_SIMT = 1, ATTN_PATH_TENSOR = 2 } attn_path_t;
+
+/*
+ * attn_fwd -- O and LSE from Q, K, V.
+ *   Q   [B,H,n,d]   K [B,H,m,d]   V [B,H,m,dv]          (read only)
+ *   O   [B,H,n,dv]  element type; LSE [B,H,n] fp32     (written)
+ *   causal != 0 masks key j > query i before the softmax and needs n == m.
+ *   scale multiplies Q K^T; the pages use 1/sqrt(d). It must be finite.
+ *   Limits: 1 <= B*H < 2^31, 1 <= n, m < 2^24, 1 <= d, dv <= 128.
+ */
+attn_status_t attn_fwd(const void* Q, const void* K, const void* V,
+                       void* O, float* LSE,
+                       int B, int H, int n, int m, int d, int dv,
+                       attn_dtype_t dtype, int causal, float scale, void* stream);
+
+/*
+ * attn_bwd_workspace_size -- bytes of device scratch that attn_bwd needs for
+ * these sizes: D = rowsum(dO * O) and the LSE in base 2, both [B,H,n] fp32
+ * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ.
+ * Returns 0 if the sizes are invalid.
+ */
+size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv,
+                               attn_dtype_t dtype);
+
+/*
+ * attn_bwd -- dQ, dK, dV from Q, K, V, O, dO and the forward's LSE.
+ *   Q, K, V, O, dO, LSE as in attn_fwd (read only); O and LSE must come
+ *   from attn_fwd on the same Q, K, V, causal and scale.
+ *   dQ [B,H,n,d], dK [B,H,m,d], dV [B,H,m,dv]  element type (written)
+ *   workspace: caller-owned device memory of at least
+ *   attn_bwd_workspace_size(...) bytes; its contents on entry do not matter
+ *   and are overwritten. It must not be in use by another call in flight.
+ *   P is rebuilt from Q, K and LSE; neither P nor the softmax Jacobian is
+ *   ever stored.
+ */
+attn_status_t attn_bwd(const void* Q, const void* K, const void* V,
+                       const void* O, const void* dO, const float* LSE,
+                       void* dQ, void* dK, void* dV,
+                       void* workspace, size_t workspace_bytes,
+                       int B, int H, int n, int m, int d, int dv,
+                       attn_dtype_t dtype, int causal, float scale, void* stream);
+
+/*
+ * attn_get_device_error -- synchronise `stream`, then report and clear the
+ * device-side error word of the current device. Every wait inside the
+ * tensor-core kernels is bounded; a wait that runs out writes
+ * ATTN_ERR_DEVICE_TIMEOUT there, and the kernel releases its tensor memory
+ * and exits instead of hanging. The word is sticky: while it is set, the
+ * tensor-core kernels skip their work, so outputs of calls made after a
+ * timeout are undefined until this function has read and cleared it.
+ * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT, or ATTN_ERR_CUDA if synchronising
+ * or reading failed.
+ */
+attn_status_t attn_get_device_error(void* stream);
+
+/*
+ * attn_probe_timeout -- launch one CTA that waits on a barrier nothing will
+ * ever complete, with a wait bound of `timeout_us` microseconds (1..10^6), so
+ * that a test can check the timeout path end to end: afterwards
+ * attn_get_device_error() must return ATTN_ERR_DEVICE_TIMEOUT.
+ */
+attn_status_t attn_probe_timeout(unsigned timeout_us, void* stream);
+
+/* Select the kernel path for later calls (see attn_path_t). */
+attn_status_t attn_set_path(attn_path_t path);
+
+/* Number of kernels the last successful attn_fwd/attn_bwd call launched. */
+int attn_last_launch_count(void);
+
+/* A static, human-readable name for a status code. */
+const char* attn_status_string(attn_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,175 @@
+"""Python binding of the B200 attention library (``libattn.so``).
+
+Argument marshalling only: each function checks that it was given contiguous
+CUDA tensors of one element type, allocates outputs with torch when the caller
+did not pass them, and calls the C entry point of the same name on torch's
+current stream. Every arithmetic step runs in the library's CUDA kernels;
+there is no fallback, and importing this package fails loudly when the
+library has not been built (``python -m scaled_dot_product_saving_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "AttnError", "LIB_PATH", "lib", "ATTN_F32", "ATTN_BF16",
+    "ATTN_PATH_AUTO", "ATTN_PATH_SIMT", "ATTN_PATH_TENSOR",
+    "attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_error",
+    "attn_probe_timeout", "attn_set_path", "attn_last_launch_count", "attn_status_string",
+    "dtype_code",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+
+ATTN_F32, ATTN_BF16 = 0, 1
+ATTN_PATH_AUTO, ATTN_PATH_SIMT, ATTN_PATH_TENSOR = 0, 1, 2
+ATTN_OK = 0
+ATTN_ERR_DEVICE_TIMEOUT = 8
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {attn_status_string(code)} (status {code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m scaled_dot_product_saving_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
+    L.attn_fwd.restype = i
+    L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                           i, i, i, i, i, i, i, i, f, vp]
+    L.attn_bwd.restype = i
+    L.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.attn_bwd_workspace_size.restype = sz
+    L.attn_get_device_error.argtypes = [vp]
+    L.attn_get_device_error.restype = i
+    L.attn_probe_timeout.argtypes = [ctypes.c_uint, vp]
+    L.attn_probe_timeout.restype = i
+    L.attn_set_path.argtypes = [i]
+    L.attn_set_path.restype = i
+    L.attn_last_launch_count.argtypes = []
+    L.attn_last_launch_count.restype = i
+    L.attn_status_string.argtypes = [i]
+    L.attn_status_string.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def attn_status_string(code: int) -> str:
+    return lib.attn_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str) -> None:
+    if code != ATTN_OK:
+        raise AttnError(code, where)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.float32:
+        return ATTN_F32
+    if dt == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"unsupported dtype {dt}; use torch.float32 or torch.bfloat16")
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dims(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("Q, K, V must be [B, H, N, d] tensors")
+    B, H, n, d = q.shape
+    if k.shape[:2] != (B, H) or v.shape[:2] != (B, H) or k.shape[3] != d or v.shape[2] != k.shape[2]:
+        raise ValueError(f"shape mismatch Q{tuple(q.shape)} K{tuple(k.shape)} V{tuple(v.shape)}")
+    return B, H, n, k.shape[2], d, v.shape[3]
+
+
+def _require(*ts):
+    dt = ts[0].dtype
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if t.dtype != dt:
+            raise TypeError("Q, K, V, O, dO must share one dtype")
+
+
+def attn_bwd_workspace_size(B, H, n, m, d, dv, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(lib.attn_bwd_workspace_size(B, H, n, m, d, dv, code))
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """Returns (O, LSE) for [B,H,N,d] CUDA tensors."""
+    _require(q, k, v)
+    B, H, n, m, d, dv = _dims(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, n, dv), dtype=q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, m, d, dv,
+                        dtype_code(q.dtype), int(bool(causal)), scale, _stream_handle(stream)),
+           "attn_fwd")
+    return out, lse
+
+
+def attn_bwd(q, k, v, o, do, lse, causal=False, scale=None, workspace=None,
+             dq=None, dk=None, dv=None, stream=None):
+    """Returns (dQ, dK, dV) with the shapes of Q, K, V."""
+    _require(q, k, v, o, do)
+    B, H, n, m, d, dvw = _dims(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    code = dtype_code(q.dtype)
+    need = attn_bwd_workspace_size(B, H, n, m, d, dvw, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if dq is None:
+        dq = torch.empty_like(q)
+    if dk is None:
+        dk = torch.empty_like(k)
+    if dv is None:
+        dv = torch.empty_like(v)
+    _check(lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                        workspace.numel() * workspace.element_size(),
+                        B, H, n, m, d, dvw, code, int(bool(causal)), scale,
+                        _stream_handle(stream)),
+           "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_get_device_error(stream=None) -> int:
+    """Synchronises the stream; returns the device status code and clears it."""
+    return int(lib.attn_get_device_error(_stream_handle(stream)))
+
+
+def attn_probe_timeout(timeout_us: int, stream=None) -> None:
+    _check(lib.attn_probe_timeout(int(timeout_us), _stream_handle(stream)), "attn_probe_timeout")
+
+
+def attn_set_path(path: int) -> None:
+    _check(lib.attn_set_path(int(path)), "attn_set_path")
+
+
+def attn_last_launch_count() -> int:
+    return int(lib.attn_last_launch_count())

@@ -1,0 +1,362 @@
+// attn.cu -- the C ABI declared in include/attn.h: argument checks, workspace
+// carving, TMA descriptors, kernel-path choice and launches. All kernels are
+// compiled into this one translation unit.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "attn.h"
+#include "sm100.cuh"
+#include "simt.cuh"
+#include "prep.cuh"
+#include "fwd_tc.cuh"
+#include "bwd_tc.cuh"
+
+namespace {
+
+constexpr unsigned long long kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTile = 128;
+
+std::atomic<int> g_path{ATTN_PATH_AUTO};
+thread_local int g_last_launches = 0;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+attn_status_t check_sizes(int B, int H, int n, int m, int d, int dv, attn_dtype_t dtype,
+                          int causal) {
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+    if (B < 1 || H < 1 || n < 1 || m < 1 || d < 1 || dv < 1) return ATTN_ERR_SHAPE;
+    if (static_cast<long long>(B) * H >= (1ll << 31)) return ATTN_ERR_SHAPE;
+    if (n >= (1 << 24) || m >= (1 << 24)) return ATTN_ERR_SHAPE;
+    if (causal && n != m) return ATTN_ERR_SHAPE;
+    if (d > attn::simt::kMaxWidth || dv > attn::simt::kMaxWidth) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+bool tensor_path_fits(attn_dtype_t dtype, int d, int dv) {
+    return dtype == ATTN_BF16 && d == dv && (d == 64 || d == 128);
+}
+
+// Decide the path; ATTN_OK and *use_tensor set, or an error.
+attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, bool* use_tensor) {
+    const int p = g_path.load();
+    const bool fits = tensor_path_fits(dtype, d, dv);
+    if (p == ATTN_PATH_TENSOR && !fits) return ATTN_ERR_UNSUPPORTED;
+    *use_tensor = fits && p != ATTN_PATH_SIMT;
+    return ATTN_OK;
+}
+
+struct Workspace {
+    size_t lse2_off, dd_off, dq_off, total;
+    int n_pad;
+};
+
+Workspace carve(int B, int H, int n, int d) {
+    Workspace w;
+    const size_t bh = static_cast<size_t>(B) * H;
+    w.n_pad = static_cast<int>(round_up(static_cast<size_t>(n), kTile));
+    const size_t row_bytes = round_up(bh * w.n_pad * sizeof(float), 256);
+    w.lse2_off = 0;
+    w.dd_off = row_bytes;
+    w.dq_off = 2 * row_bytes;
+    w.total = w.dq_off + round_up(bh * static_cast<size_t>(n) * d * sizeof(float), 256);
+    return w;
+}
+
+// ---------------------------------------------------------------- TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [BH, rows, width] bf16 viewed as 3-D (width innermost); boxes of 64 x 128 x 1
+// with the 128-byte swizzle the UMMA descriptors expect.
+bool make_map(CUtensorMap* map, const void* base, int width, int rows, int bh) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(width) * 2,
+                             static_cast<cuuint64_t>(width) * 2 * rows};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int grid_for(size_t work_items, int per_block, int cap) {
+    size_t g = (work_items + per_block - 1) / per_block;
+    if (g < 1) g = 1;
+    if (g > static_cast<size_t>(cap)) g = cap;
+    return static_cast<int>(g);
+}
+
+template <typename T>
+attn_status_t fwd_simt(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH,
+                       int n, int m, int d, int dv, int causal, float scale, cudaStream_t st) {
+    const size_t smem = attn::simt::fwd_smem_bytes<T>(d, dv);
+    auto kern = attn::simt::fwd_kernel<T>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    dim3 grid((n + attn::simt::kTile - 1) / attn::simt::kTile, BH);
+    kern<<<grid, attn::simt::kThreads, smem, st>>>(
+        static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
+        static_cast<T*>(O), LSE, n, m, d, dv, causal, scale);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         int BH, int n, int m, int causal, float scale, cudaStream_t st) {
+    using C = attn::fwdtc::Cfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) || !make_map(&mv, V, D, m, BH))
+        return ATTN_ERR_CUDA;
+    auto kern = attn::fwdtc::fwd_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const long long grid = static_cast<long long>((n + kTile - 1) / kTile) * BH;
+    kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
+        mq, mk, mv, static_cast<__nv_bfloat16*>(O), LSE, n, m, BH, causal, scale * kLog2e,
+        kWaitBudgetNs);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T>
+attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float* lse2, float* Dd,
+                         float* dQacc, int BH, int n, int n_pad, int d, int dv, cudaStream_t st) {
+    const size_t rows = static_cast<size_t>(BH) * n_pad;
+    const size_t dq_elems = static_cast<size_t>(BH) * n * d;
+    const bool vec = sizeof(T) == 2 && dv % 8 == 0 && (dv / 8) <= 32 && 32 % (dv / 8) == 0 &&
+                     dq_elems % 4 == 0;
+    if (vec) {
+        const int rows_per_block = (attn::prep::kThreads / 32) * (32 / (dv / 8));
+        const int grid = grid_for(rows, rows_per_block, 148 * 16);
+        attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
+            lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv);
+    } else {
+        const int grid = grid_for(rows, attn::prep::kThreads / 32, 148 * 16);
+        attn::prep::preprocess_generic<T><<<grid, attn::prep::kThreads, 0, st>>>(
+            static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, dq_elems,
+            BH, n, n_pad, dv);
+    }
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T>
+attn_status_t finalize(const float* dQacc, void* dQ, size_t elems, float post_scale,
+                       cudaStream_t st) {
+    const int grid = grid_for(elems / 4 + 1, attn::prep::kThreads, 148 * 16);
+    attn::prep::finalize_dq<T><<<grid, attn::prep::kThreads, 0, st>>>(
+        dQacc, static_cast<T*>(dQ), elems, post_scale);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T>
+attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* dO,
+                       const float* LSE, const float* Dd, int n_pad, float* dQacc, void* dK,
+                       void* dV, int BH, int n, int m, int d, int dv, int causal, float scale,
+                       cudaStream_t st) {
+    const size_t smem = attn::simt::bwd_smem_bytes<T>(d, dv);
+    auto kern = attn::simt::bwd_kernel<T>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    dim3 grid((m + attn::simt::kTile - 1) / attn::simt::kTile, BH);
+    kern<<<grid, attn::simt::kThreads, smem, st>>>(
+        static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
+        static_cast<const T*>(dO), LSE, Dd, n_pad, dQacc, static_cast<T*>(dK),
+        static_cast<T*>(dV), n, m, d, dv, causal, scale);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void* dO,
+                         const float* lse2, const float* Dd, int n_pad, float* dQacc, void* dK,
+                         void* dV, int BH, int n, int m, int causal, float scale,
+                         cudaStream_t st) {
+    using C = attn::bwdtc::Cfg<D>;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) ||
+        !make_map(&mv, V, D, m, BH) || !make_map(&mdo, dO, D, n, BH))
+        return ATTN_ERR_CUDA;
+    auto kern = attn::bwdtc::bwd_kernel<D>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const long long grid = static_cast<long long>((m + kTile - 1) / kTile) * BH;
+    kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
+        mq, mk, mv, mdo, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
+        static_cast<__nv_bfloat16*>(dV), n, m, BH, causal, scale, scale * kLog2e, kWaitBudgetNs);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+__global__ void probe_timeout_kernel(unsigned long long budget_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort;
+    if (threadIdx.x == 0) {
+        abort = 0;
+        attn::mbar_init(&bar, 1);
+        attn::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // Nothing ever arrives on `bar`: the wait must give up after budget_ns.
+        if (!attn::mbar_wait(&bar, 0, &abort, budget_ns))
+            attn::record_device_error(attn::kErrTimeout);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_set_path(attn_path_t path) {
+    if (path != ATTN_PATH_AUTO && path != ATTN_PATH_SIMT && path != ATTN_PATH_TENSOR)
+        return ATTN_ERR_UNSUPPORTED;
+    g_path.store(path);
+    return ATTN_OK;
+}
+
+int attn_last_launch_count(void) { return g_last_launches; }
+
+size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv, attn_dtype_t dtype) {
+    if (check_sizes(B, H, n, m, d, dv, dtype, 0) != ATTN_OK) return 0;
+    return carve(B, H, n, d).total;
+}
+
+attn_status_t attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                       int H, int n, int m, int d, int dv, attn_dtype_t dtype, int causal,
+                       float scale, void* stream) {
+    attn_status_t s = check_sizes(B, H, n, m, d, dv, dtype, causal);
+    if (s != ATTN_OK) return s;
+    if (!std::isfinite(scale)) return ATTN_ERR_SHAPE;
+    if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+        return ATTN_ERR_ALIGN;
+    bool tensor = false;
+    if ((s = choose_path(dtype, d, dv, &tensor)) != ATTN_OK) return s;
+    const int BH = B * H;
+    cudaStream_t st = as_stream(stream);
+    if (tensor)
+        s = (d == 64) ? fwd_tensor<64>(Q, K, V, O, LSE, BH, n, m, causal, scale, st)
+                      : fwd_tensor<128>(Q, K, V, O, LSE, BH, n, m, causal, scale, st);
+    else if (dtype == ATTN_F32)
+        s = fwd_simt<float>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+    else
+        s = fwd_simt<__nv_bfloat16>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+    if (s == ATTN_OK) g_last_launches = 1;
+    return s;
+}
+
+attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* O,
+                       const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                       void* workspace, size_t workspace_bytes, int B, int H, int n, int m, int d,
+                       int dv, attn_dtype_t dtype, int causal, float scale, void* stream) {
+    attn_status_t s = check_sizes(B, H, n, m, d, dv, dtype, causal);
+    if (s != ATTN_OK) return s;
+    if (!std::isfinite(scale)) return ATTN_ERR_SHAPE;
+    if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return ATTN_ERR_NULL;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
+        !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+        return ATTN_ERR_ALIGN;
+    const Workspace w = carve(B, H, n, d);
+    if (!workspace || workspace_bytes < w.total) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+    bool tensor = false;
+    if ((s = choose_path(dtype, d, dv, &tensor)) != ATTN_OK) return s;
+
+    const int BH = B * H;
+    cudaStream_t st = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
+    float* Dd = reinterpret_cast<float*>(ws + w.dd_off);
+    float* dQacc = reinterpret_cast<float*>(ws + w.dq_off);
+    const size_t dq_elems = static_cast<size_t>(BH) * n * d;
+
+    s = (dtype == ATTN_F32)
+            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, st)
+            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, st);
+    if (s != ATTN_OK) return s;
+    if (tensor) {
+        s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, w.n_pad, dQacc, dK, dV, BH, n, m,
+                                       causal, scale, st)
+                      : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, w.n_pad, dQacc, dK, dV, BH, n, m,
+                                        causal, scale, st);
+        if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, 1.0f, st);
+    } else if (dtype == ATTN_F32) {
+        s = bwd_simt<float>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv, causal,
+                            scale, st);
+        if (s == ATTN_OK) s = finalize<float>(dQacc, dQ, dq_elems, scale, st);
+    } else {
+        s = bwd_simt<__nv_bfloat16>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv,
+                                    causal, scale, st);
+        if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, scale, st);
+    }
+    if (s == ATTN_OK) g_last_launches = 3;
+    return s;
+}
+
+attn_status_t attn_get_device_error(void* stream) {
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, attn::g_device_error, sizeof(v)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(attn::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        return ATTN_ERR_DEVICE_TIMEOUT;
+    }
+    return ATTN_OK;
+}
+
+attn_status_t attn_probe_timeout(unsigned timeout_us, void* stream) {
+    if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_SHAPE;
+    probe_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(1000ull * timeout_us);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+const char* attn_status_string(attn_status_t s) {
+    switch (s) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_NULL: return "null pointer";
+        case ATTN_ERR_SHAPE: return "invalid size or scale (or causal with n != m)";
+        case ATTN_ERR_DTYPE: return "unknown dtype";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported by this build";
+        case ATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case ATTN_ERR_CUDA: return "CUDA runtime error";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

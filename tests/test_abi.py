@@ -1,0 +1,120 @@
+"""The C ABI on the CPU: the library builds, loads, exports every function the
+header declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from scaled_dot_product_saving_b200 import build
+    build.build()
+    import scaled_dot_product_saving_b200 as m
+    return m
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_size",
+                     "attn_get_device_error", "attn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_function(L):
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+# Fake, aligned, non-null device addresses: validation must reject the calls
+# below before any of them is used.
+P = ctypes.c_void_p(0x10000)
+MIS = ctypes.c_void_p(0x10008)
+NUL = ctypes.c_void_p(0)
+
+
+def fwd(L, q=P, k=P, v=P, o=P, lse=P, B=1, H=1, n=64, m=64, d=64, dv=64, dt=1, causal=0,
+        scale=0.125):
+    return L.lib.attn_fwd(q, k, v, o, lse, B, H, n, m, d, dv, dt, causal, scale, NUL)
+
+
+def bwd(L, ws=P, wsb=1 << 40, q=P, B=1, H=1, n=64, m=64, d=64, dv=64, dt=1, causal=0,
+        scale=0.125, dq=P):
+    return L.lib.attn_bwd(q, P, P, P, P, P, dq, P, P, ws, wsb, B, H, n, m, d, dv, dt, causal,
+                          scale, NUL)
+
+
+def test_argument_checks_forward(L):
+    assert fwd(L, q=NUL) == 1
+    assert fwd(L, lse=NUL) == 1
+    assert fwd(L, B=0) == 2
+    assert fwd(L, n=0) == 2
+    assert fwd(L, n=64, m=65, causal=1) == 2          # causal needs n == m
+    assert fwd(L, n=1 << 24, m=1 << 24) == 2
+    assert fwd(L, dt=7) == 3
+    assert fwd(L, d=129) == 4
+    assert fwd(L, q=MIS) == 5
+    assert fwd(L, scale=float("nan")) == 2
+    assert fwd(L, scale=float("inf")) == 2
+
+
+def test_argument_checks_backward(L):
+    assert bwd(L, q=NUL) == 1
+    assert bwd(L, dq=NUL) == 1
+    assert bwd(L, n=63, causal=1) == 2
+    assert bwd(L, dt=2) == 3
+    assert bwd(L, dv=200) == 4
+    assert bwd(L, q=MIS) == 5
+    assert bwd(L, ws=NUL) == 6
+    need = L.attn_bwd_workspace_size(1, 1, 64, 64, 64, 64, 1)
+    assert bwd(L, wsb=need - 1) == 6
+    assert bwd(L, ws=MIS, wsb=need) == 5
+
+
+def test_tensor_path_request_rejects_other_shapes(L):
+    try:
+        L.attn_set_path(L.ATTN_PATH_TENSOR)
+        assert fwd(L, dt=0) == 4          # fp32 has no tensor-core path
+        assert fwd(L, d=32, dv=32) == 4
+        assert fwd(L, d=64, dv=128) == 4
+    finally:
+        L.attn_set_path(L.ATTN_PATH_AUTO)
+    assert L.lib.attn_set_path(9) == 4
+
+
+def test_workspace_size_formula(L):
+    def expect(B, H, n, d):
+        bh = B * H
+        n_pad = -(-n // 128) * 128
+        rows = -(-(bh * n_pad * 4) // 256) * 256
+        return 2 * rows + -(-(bh * n * d * 4) // 256) * 256
+    for (B, H, n, m, d) in [(1, 1, 1, 1, 1), (4, 16, 1024, 1024, 64), (2, 32, 4096, 4096, 128),
+                            (8, 16, 512, 2048, 64), (1, 3, 77, 90, 40)]:
+        assert L.attn_bwd_workspace_size(B, H, n, m, d, d, 1) == expect(B, H, n, d)
+    assert L.attn_bwd_workspace_size(0, 1, 1, 1, 1, 1, 1) == 0
+    assert L.attn_bwd_workspace_size(1, 1, 1, 1, 300, 1, 1) == 0
+
+
+def test_status_strings(L):
+    for code in range(9):
+        s = L.attn_status_string(code)
+        assert s and s != "unknown status"
+    assert L.attn_status_string(99) == "unknown status"
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_valid_call_without_a_device_reports_cuda_error(L):
+    assert fwd(L) == 7
+    assert fwd(L, dt=0) == 7

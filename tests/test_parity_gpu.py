@@ -1,0 +1,104 @@
+"""GPU parity: the CUDA path against the float64 oracle on the same seeded
+inputs, through the C ABI. Tolerance: max|gpu - ref| / max|ref| per output
+tensor, 1e-5 for fp32 inputs and 2e-2 for bf16 inputs (fp32 accumulation)."""
+import pytest
+import torch
+
+import synth
+from parity_util import TOL, full_compare, sampled_compare
+
+pytestmark = pytest.mark.gpu
+
+lib = pytest.importorskip("scaled_dot_product_saving_b200")
+
+
+@pytest.fixture(autouse=True)
+def _auto_path():
+    lib.attn_set_path(lib.ATTN_PATH_AUTO)
+    yield
+    lib.attn_set_path(lib.ATTN_PATH_AUTO)
+
+
+def _assert_within(errs, tol, label):
+    bad = {k: v for k, v in errs.items() if not v <= tol}
+    assert not bad, f"{label}: {errs}"
+
+
+# ----------------------------------------------------------------------------
+# The single-head fp32 workload, compared in full
+# ----------------------------------------------------------------------------
+def test_single_head_f32_64():
+    w = synth.workload("single_head_f32_64")
+    _assert_within(full_compare(w), TOL["f32"], w.name)
+
+
+# ----------------------------------------------------------------------------
+# Small and edge shapes, compared in full. bf16 with d == dv in {64, 128}
+# runs on the tensor cores; the others on the CUDA-core path.
+# ----------------------------------------------------------------------------
+SMALL = [
+    # B, H, n, m, d, dv, dtype, causal, std_qk
+    (1, 2, 384, 384, 64, 64, "bf16", True, 1.0),      # several tiles, causal
+    (1, 2, 384, 384, 128, 128, "bf16", True, 1.0),
+    (2, 1, 128, 128, 128, 128, "bf16", False, 1.0),   # exactly one tile
+    (1, 2, 300, 300, 128, 128, "bf16", True, 1.0),    # ragged tail, causal
+    (1, 2, 200, 520, 64, 64, "bf16", False, 1.0),     # n != m, both ragged
+    (1, 1, 130, 1, 128, 128, "bf16", False, 1.0),     # a single key
+    (1, 1, 1, 700, 64, 64, "bf16", False, 1.0),       # a single query
+    (1, 1, 1, 1, 64, 64, "bf16", True, 1.0),          # n = m = 1
+    (1, 2, 256, 1024, 64, 64, "bf16", False, 3.0),    # large scores, stable LSE
+    (1, 1, 513, 513, 128, 128, "bf16", True, 1.0),    # one row past a tile
+    (1, 2, 100, 100, 40, 40, "bf16", True, 1.0),      # CUDA-core path widths
+    (1, 1, 70, 90, 32, 48, "bf16", False, 1.0),
+    (2, 2, 77, 77, 24, 24, "f32", True, 1.0),
+    (1, 1, 129, 65, 128, 96, "f32", False, 2.0),
+]
+
+
+@pytest.mark.parametrize("B,H,n,m,d,dv,dt,causal,std", SMALL)
+def test_small_shapes(B, H, n, m, d, dv, dt, causal, std):
+    w = synth.make_small(B, H, n, m, d, dv, dt, causal, seed=B * 1000 + n + m + d, std_qk=std)
+    _assert_within(full_compare(w), TOL[dt], w.name)
+
+
+@pytest.mark.parametrize("d,causal", [(64, True), (128, False)])
+def test_cuda_core_path_bf16(d, causal):
+    """The CUDA-core path forced on shapes the tensor cores would take."""
+    lib.attn_set_path(lib.ATTN_PATH_SIMT)
+    w = synth.make_small(1, 2, 200, 200, d, d, "bf16", causal, seed=11)
+    _assert_within(full_compare(w), TOL["bf16"], w.name)
+
+
+def test_tensor_path_is_taken():
+    lib.attn_set_path(lib.ATTN_PATH_TENSOR)
+    w = synth.make_small(1, 1, 256, 256, 64, 64, "bf16", True, seed=3)
+    _assert_within(full_compare(w), TOL["bf16"], w.name)
+    assert lib.attn_last_launch_count() == 3
+
+
+# ----------------------------------------------------------------------------
+# The four bf16 workloads at full size, in the launch configuration the
+# benchmark times: sampled rows against the oracle, invariants over all heads.
+# ----------------------------------------------------------------------------
+FULL = ["causal_b4h16_n1024_d64", "causal_b2h32_n4096_d128",
+        "cross_b8h16_n512_m2048_d64", "causal_b1h32_n16384_d128"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled(name):
+    w = synth.workload(name)
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    errs, inv = sampled_compare(w, heads)
+    _assert_within(errs, TOL["bf16"], name)
+    _assert_within(inv, TOL["bf16"], name + " invariants")
+
+
+def test_timeout_path_reports_error():
+    """A bounded wait that nothing completes must come back as an error
+    status, with the context still usable afterwards."""
+    assert lib.attn_get_device_error() == 0
+    lib.attn_probe_timeout(2000)
+    assert lib.attn_get_device_error() == lib.ATTN_ERR_DEVICE_TIMEOUT
+    assert lib.attn_get_device_error() == 0
+    w = synth.make_small(1, 1, 128, 128, 64, 64, "bf16", False, seed=5)
+    _assert_within(full_compare(w), TOL["bf16"], "after timeout")
