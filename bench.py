@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Attention backward throughput on B200: one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+attn_fwd (O and LSE) followed by attn_bwd (dQ, dK, dV). The metric is the
+backward's counted FLOPs (2.5x the forward's two matmuls, 4*B*H*n*m*d, halved
+when causal) over the backward's device time, in TFLOP/s, summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the float64 CPU oracle, timed
+
+With N > 1 the script runs under torch.distributed.run, one rank per GPU; the
+(batch, head) problems are independent, so every rank runs the same workload
+on its own seeded data with no collective on the data path ("weak" scaling),
+and the timed region is bracketed by barriers and reduced as a max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "causal_b2h32_n4096_d128"
+METRIC = "attn backward TFLOP/s (bf16, causal) and % of B200 dense-BF16 tensor peak"
+L2_BYTES = 126 * 1024 * 1024
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "bwd_tc_causal_b2h32_n4096_d128.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "scaled_dot_product_saving_b200", "csrc", f)
+                  for f in ("bwd_tc.cuh", "sm100.cuh")]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=8)
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if a.steps < 1:
+        p.error("--steps must be >= 1")
+    return a
+
+
+# ---------------------------------------------------------------- helpers
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the backward kernel from the committed ncu
+    summary, or None when it is missing, for another workload, or taken on a
+    kernel source that has changed since."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            fields = dict(line.split(":", 1) for line in f if ":" in line)
+    except OSError:
+        return None
+    fields = {k.strip(): v.strip() for k, v in fields.items()}
+    if fields.get("workload") != workload or fields.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def counted_bwd_flops_per_head(w: synth.Workload) -> float:
+    return w.bwd_flops() / (w.B * w.H)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                mask = get(self.handle)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- multi-rank
+def init_distributed():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise max of a list of floats over all ranks."""
+    if world == 1:
+        return list(values)
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate(per_rank_flops, local_ms, world, device):
+    """Whole-job throughput: all ranks' FLOPs over the slowest rank's time."""
+    (slowest_ms,) = max_over_ranks([local_ms], world, device)
+    return world * per_rank_flops / (slowest_ms * 1e-3) / 1e12, slowest_ms
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, w, rank, world, local):
+    import scaled_dot_product_saving_b200 as lib
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q, k, v, do = (t.to(dev) for t in synth.make_inputs(w, seed=w.seed + 1000 * rank))
+    o = torch.empty((w.B, w.H, w.n, w.dv), dtype=q.dtype, device=dev)
+    lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(lib.attn_bwd_workspace_size(w.B, w.H, w.n, w.m, w.d, w.dv, q.dtype),
+                     dtype=torch.uint8, device=dev)
+    working_set = sum(t.numel() * t.element_size() for t in (q, k, v, o, do, dq, dk, dv, ws))
+    flush = None
+    if working_set < 2 * L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if flush is not None:
+            flush.zero_()
+        if evs:
+            evs[0].record()
+        lib.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        if evs:
+            evs[1].record()
+        lib.attn_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws,
+                     dq=dq, dk=dk, dv=dv)
+        if evs:
+            evs[2].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if lib.attn_get_device_error() != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    sampler.start()
+    lib.attn_trace_begin(min(65536, 8 * args.steps))
+    t_start.record()
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world, local)
+    sampler.stop()
+    trace = lib.attn_trace_end()
+    if lib.attn_get_device_error() != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    bwd_sum, fwd_sum = sum(bwd_ms), sum(fwd_ms)
+    slow_total, slow_bwd, slow_fwd = max_over_ranks([total_ms, bwd_sum, fwd_sum], world, dev)
+    value = world * args.steps * w.bwd_flops() / (slow_bwd * 1e-3) / 1e12
+
+    by_kernel = {}
+    for name, ms in trace:
+        by_kernel.setdefault(name, []).append(ms)
+    main = "bwd_tensor" if "bwd_tensor" in by_kernel else "bwd_simt"
+    main_ms = statistics.mean(by_kernel[main])
+    peaks, peaks_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = w.bwd_flops() / (main_ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    pin = [t.to("cpu").pin_memory() for t in (q, k, v, do)]
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in pin)
+    d2h = sum(t.numel() * t.element_size() for t in outs_host)
+    e2e_ms = []
+    for i in range(args.e2e_steps + 2 if args.e2e_steps > 0 else 0):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for src, dst in zip(pin, (q, k, v, do)):
+            dst.copy_(src, non_blocking=True)
+        lib.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        lib.attn_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws,
+                     dq=dq, dk=dk, dv=dv)
+        for src, dst in zip((dq, dk, dv), outs_host):
+            dst.copy_(src, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    if e2e_ms:
+        (slow_e2e,) = max_over_ranks([sum(e2e_ms)], world, dev)
+        e2e = {"value": round(world * len(e2e_ms) * w.bwd_flops() / (slow_e2e * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(slow_e2e / len(e2e_ms), 4)}
+    else:
+        e2e = None
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(slow_total / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": w.B, "H": w.H, "n": w.n, "m": w.m, "d": w.d, "dv": w.dv,
+            "causal": w.causal, "scale": w.scale,
+            "parallelism": "replicas" if world == 1 else f"independent (batch, head) problems x{world}",
+            "l2": ("flushed between steps (256 MiB write)" if flush is not None else
+                   f"inputs larger than L2 ({working_set / 2**20:.0f} MiB per step)"),
+        },
+        "fwd_ms": round(slow_fwd / args.steps, 4),
+        "bwd_ms": round(slow_bwd / args.steps, 4),
+        "fwd_tflops": round(world * args.steps * w.fwd_flops() / (slow_fwd * 1e-3) / 1e12, 3),
+        "frac_of_datasheet_bf16": round(value / world / DATASHEET_BF16_TFLOPS, 4),
+        "kernel_ms": {k2: round(statistics.mean(v2), 4) for k2, v2 in by_kernel.items()},
+        "roofline": {
+            "bound": "tensor", "kernel": main, "achieved": round(achieved, 3),
+            "peak": peak, "peak_source": f"bf16_tflops ({peaks_src}, burst)",
+            "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(w.name),
+        },
+        "e2e": e2e,
+        "gpu_launches": len(trace),
+        "clocks": sampler.summary(),
+    }
+    return result
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample(w, seconds, max_heads=None):
+    """Time the oracle backward on whole heads of the workload until `seconds`
+    have passed. Returns (TFLOP/s in the metric's counting, heads, elapsed)."""
+    import oracle.ref as ref
+    q, k, v, do = synth.make_inputs(w)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    done, t0 = 0, time.perf_counter()
+    while True:
+        b, h = heads[done % len(heads)]
+        Q, K, V, dO = (t[b, h].to(torch.float64).numpy() for t in (q, k, v, do))
+        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale)
+        done += 1
+        elapsed = time.perf_counter() - t0
+        if elapsed >= seconds or (max_heads and done >= max_heads):
+            break
+    return done * counted_bwd_flops_per_head(w) / elapsed / 1e12, done, elapsed
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return None
+    import oracle.ref as ref
+    q, k, v, do = synth.make_inputs(w)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+
+    def one(i):
+        b, h = heads[i % len(heads)]
+        Q, K, V, dO = (t[b, h].to(torch.float64).numpy() for t in (q, k, v, do))
+        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        one(i)
+    elapsed = time.perf_counter() - t0
+    value = args.steps * counted_bwd_flops_per_head(w) / elapsed / 1e12
+    cores = blas_threads()
+    sample = (f"one (batch, head) problem of {w.name} per step "
+              f"(n={w.n}, m={w.m}, d={w.d}), float64 oracle backward")
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * elapsed / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "m": w.m, "d": w.d,
+                   "dv": w.dv, "causal": w.causal, "scale": w.scale},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    w = synth.workload(args.workload)
+    rank, world, local = init_distributed()
+    try:
+        if args.impl == "reference":
+            out = run_reference(args, w, rank, world)
+        else:
+            out = run_ours(args, w, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                tf, nheads, secs = oracle_sample(w, args.cpu_seconds)
+                out["cpu_baseline"] = {
+                    "value": tf, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                    "sample": f"{nheads} (batch, head) problems of {w.name} through the float64 "
+                              f"oracle backward in {secs:.1f} s"}
+            elif rank == 0:
+                out["cpu_baseline"] = None
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

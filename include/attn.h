@@ -127,6 +127,34 @@ attn_status_t attn_get_device_error(void* stream);
  */
 attn_status_t attn_probe_timeout(unsigned timeout_us, void* stream);
 
+/*
+ * Kernel tracing. Between attn_trace_begin and attn_trace_end, every kernel
+ * that attn_fwd/attn_bwd launch from the calling host thread is bracketed by
+ * a pair of CUDA events on the call's stream (at most `capacity` launches,
+ * 1..65536, are recorded; later ones run untraced). attn_trace_end stops
+ * recording, waits for the recorded events, and writes up to `max_entries`
+ * (kernel id, milliseconds) pairs in launch order to `out` (which may be NULL
+ * when max_entries is 0). It returns the number of launches recorded, or -1
+ * if the CUDA runtime failed. The events are created on first use and reused;
+ * no device memory is allocated.
+ */
+typedef enum {
+    ATTN_KERNEL_FWD_TENSOR = 1,   /* tcgen05 forward                          */
+    ATTN_KERNEL_FWD_SIMT = 2,     /* CUDA-core forward                        */
+    ATTN_KERNEL_PREPROCESS = 3,   /* D = rowsum(dO*O), base-2 LSE, zero dQacc */
+    ATTN_KERNEL_BWD_TENSOR = 4,   /* tcgen05 backward                         */
+    ATTN_KERNEL_BWD_SIMT = 5,     /* CUDA-core backward                       */
+    ATTN_KERNEL_FINALIZE = 6      /* dQ accumulator -> dQ                      */
+} attn_kernel_id_t;
+
+typedef struct {
+    int kernel;    /* attn_kernel_id_t */
+    float ms;      /* device time between the bracketing events */
+} attn_kernel_time_t;
+
+attn_status_t attn_trace_begin(int capacity);
+int attn_trace_end(attn_kernel_time_t* out, int max_entries);
+
 /* Select the kernel path for later calls (see attn_path_t). */
 attn_status_t attn_set_path(attn_path_t path);
 

@@ -59,7 +59,7 @@ import numpy as np
 __all__ = [
     "default_scale", "scores", "apply_causal_mask", "row_softmax",
     "grad_v", "grad_p", "softmax_jvp", "grad_q", "grad_k",
-    "head_forward", "head_backward", "head_backward_sampled",
+    "head_forward", "head_backward",
     "attention_forward", "attention_backward",
 ]
 
@@ -185,42 +185,6 @@ def head_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
         dQ[r0:r1] = grad_q(dS, K, scale)
         dK += grad_k(dS, Q[r0:r1], scale)
     return dQ, dK, dV
-
-
-def head_backward_sampled(Q, K, V, dO, q_rows, k_rows, causal=False,
-                          scale=None, row_block=ROW_BLOCK):
-    """Selected rows of O, lse, dQ (query rows) and of dK, dV (key rows).
-
-    The same steps as head_forward/head_backward. dQ row i needs only query
-    row i's block; dK and dV rows j need column j of P and dS over every
-    query row, so every block is still visited, but only the selected
-    columns enter the two key-side products.
-    """
-    Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, dO))
-    _check_head(Q, K, V, causal)
-    scale = default_scale(Q.shape[1]) if scale is None else float(scale)
-    q_rows = np.asarray(q_rows, dtype=np.int64)
-    k_rows = np.asarray(k_rows, dtype=np.int64)
-    n = Q.shape[0]
-    O_s = np.empty((len(q_rows), V.shape[1]))
-    lse_s = np.empty(len(q_rows))
-    dQ_s = np.empty((len(q_rows), Q.shape[1]))
-    dK_s = np.zeros((len(k_rows), K.shape[1]))
-    dV_s = np.zeros((len(k_rows), V.shape[1]))
-    for r0 in range(0, n, row_block):
-        r1 = min(n, r0 + row_block)
-        P, lse = _block_probs(Q, K, r0, r1, causal, scale)
-        dP = grad_p(dO[r0:r1], V)
-        dS = softmax_jvp(P, dP)
-        dV_s += grad_v(P[:, k_rows], dO[r0:r1])
-        dK_s += grad_k(dS[:, k_rows], Q[r0:r1], scale)
-        sel = np.nonzero((q_rows >= r0) & (q_rows < r1))[0]
-        if len(sel):
-            loc = q_rows[sel] - r0
-            O_s[sel] = P[loc] @ V
-            lse_s[sel] = lse[loc]
-            dQ_s[sel] = grad_q(dS[loc], K, scale)
-    return O_s, lse_s, dQ_s, dK_s, dV_s
 
 
 # --------------------------------------------------------------------------

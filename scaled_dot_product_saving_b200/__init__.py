@@ -20,7 +20,7 @@ __all__ = [
     "ATTN_PATH_AUTO", "ATTN_PATH_SIMT", "ATTN_PATH_TENSOR",
     "attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_error",
     "attn_probe_timeout", "attn_set_path", "attn_last_launch_count", "attn_status_string",
-    "dtype_code",
+    "dtype_code", "attn_trace_begin", "attn_trace_end", "KERNEL_NAMES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
@@ -29,6 +29,13 @@ ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_PATH_AUTO, ATTN_PATH_SIMT, ATTN_PATH_TENSOR = 0, 1, 2
 ATTN_OK = 0
 ATTN_ERR_DEVICE_TIMEOUT = 8
+
+KERNEL_NAMES = {1: "fwd_tensor", 2: "fwd_simt", 3: "preprocess", 4: "bwd_tensor",
+                5: "bwd_simt", 6: "finalize"}
+
+
+class _KernelTime(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int), ("ms", ctypes.c_float)]
 
 
 class AttnError(RuntimeError):
@@ -61,6 +68,10 @@ def _load() -> ctypes.CDLL:
     L.attn_last_launch_count.restype = i
     L.attn_status_string.argtypes = [i]
     L.attn_status_string.restype = ctypes.c_char_p
+    L.attn_trace_begin.argtypes = [i]
+    L.attn_trace_begin.restype = i
+    L.attn_trace_end.argtypes = [ctypes.POINTER(_KernelTime), i]
+    L.attn_trace_end.restype = i
     return L
 
 
@@ -173,3 +184,18 @@ def attn_set_path(path: int) -> None:
 
 def attn_last_launch_count() -> int:
     return int(lib.attn_last_launch_count())
+
+
+def attn_trace_begin(capacity: int = 4096) -> None:
+    """Start bracketing every launch of this thread with CUDA events."""
+    _check(lib.attn_trace_begin(int(capacity)), "attn_trace_begin")
+
+
+def attn_trace_end(max_entries: int = 65536):
+    """Stop tracing; returns [(kernel name, milliseconds), ...] in launch order."""
+    buf = (_KernelTime * max_entries)()
+    count = lib.attn_trace_end(buf, max_entries)
+    if count < 0:
+        raise AttnError(7, "attn_trace_end")
+    return [(KERNEL_NAMES.get(buf[k].kernel, str(buf[k].kernel)), float(buf[k].ms))
+            for k in range(min(count, max_entries))]

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -108,6 +109,46 @@ bool make_map(CUtensorMap* map, const void* base, int width, int rows, int bh) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------- tracing
+struct TraceEntry {
+    int kernel;
+    cudaEvent_t start, stop;
+};
+struct TraceState {
+    bool on = false;
+    int capacity = 0;
+    std::vector<TraceEntry> entries;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;   // reused across sessions
+};
+thread_local TraceState g_trace;
+
+// Launch through `launch()`, bracketed by events when tracing is on.
+template <typename F>
+attn_status_t traced(int kernel, cudaStream_t st, F&& launch) {
+    TraceState& t = g_trace;
+    if (!t.on || static_cast<int>(t.entries.size()) >= t.capacity) return launch();
+    const size_t k = t.entries.size();
+    if (k == t.pool.size()) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return launch();
+        if (cudaEventCreate(&b) != cudaSuccess) {
+            cudaEventDestroy(a);
+            return launch();
+        }
+        t.pool.emplace_back(a, b);
+    }
+    TraceEntry e{kernel, t.pool[k].first, t.pool[k].second};
+    cudaEventRecord(e.start, st);
+    const attn_status_t s = launch();
+    cudaEventRecord(e.stop, st);
+    t.entries.push_back(e);
+    return s;
+}
+
+inline attn_status_t launched() {
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 int grid_for(size_t work_items, int per_block, int cap) {
     size_t g = (work_items + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -124,10 +165,12 @@ attn_status_t fwd_simt(const void* Q, const void* K, const void* V, void* O, flo
                              static_cast<int>(smem)) != cudaSuccess)
         return ATTN_ERR_CUDA;
     dim3 grid((n + attn::simt::kTile - 1) / attn::simt::kTile, BH);
-    kern<<<grid, attn::simt::kThreads, smem, st>>>(
-        static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
-        static_cast<T*>(O), LSE, n, m, d, dv, causal, scale);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_FWD_SIMT, st, [&] {
+        kern<<<grid, attn::simt::kThreads, smem, st>>>(
+            static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
+            static_cast<T*>(O), LSE, n, m, d, dv, causal, scale);
+        return launched();
+    });
 }
 
 template <int D>
@@ -142,10 +185,12 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
         cudaSuccess)
         return ATTN_ERR_CUDA;
     const long long grid = static_cast<long long>((n + kTile - 1) / kTile) * BH;
-    kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
-        mq, mk, mv, static_cast<__nv_bfloat16*>(O), LSE, n, m, BH, causal, scale * kLog2e,
-        kWaitBudgetNs);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_FWD_TENSOR, st, [&] {
+        kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
+            mq, mk, mv, static_cast<__nv_bfloat16*>(O), LSE, n, m, BH, causal, scale * kLog2e,
+            kWaitBudgetNs);
+        return launched();
+    });
 }
 
 template <typename T>
@@ -158,25 +203,31 @@ attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float*
     if (vec) {
         const int rows_per_block = (attn::prep::kThreads / 32) * (32 / (dv / 8));
         const int grid = grid_for(rows, rows_per_block, 148 * 16);
-        attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
-            lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv);
-    } else {
-        const int grid = grid_for(rows, attn::prep::kThreads / 32, 148 * 16);
+        return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
+            attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
+                lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv);
+            return launched();
+        });
+    }
+    const int grid = grid_for(rows, attn::prep::kThreads / 32, 148 * 16);
+    return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
         attn::prep::preprocess_generic<T><<<grid, attn::prep::kThreads, 0, st>>>(
             static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, dq_elems,
             BH, n, n_pad, dv);
-    }
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+        return launched();
+    });
 }
 
 template <typename T>
 attn_status_t finalize(const float* dQacc, void* dQ, size_t elems, float post_scale,
                        cudaStream_t st) {
     const int grid = grid_for(elems / 4 + 1, attn::prep::kThreads, 148 * 16);
-    attn::prep::finalize_dq<T><<<grid, attn::prep::kThreads, 0, st>>>(
-        dQacc, static_cast<T*>(dQ), elems, post_scale);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_FINALIZE, st, [&] {
+        attn::prep::finalize_dq<T><<<grid, attn::prep::kThreads, 0, st>>>(
+            dQacc, static_cast<T*>(dQ), elems, post_scale);
+        return launched();
+    });
 }
 
 template <typename T>
@@ -190,11 +241,13 @@ attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* 
                              static_cast<int>(smem)) != cudaSuccess)
         return ATTN_ERR_CUDA;
     dim3 grid((m + attn::simt::kTile - 1) / attn::simt::kTile, BH);
-    kern<<<grid, attn::simt::kThreads, smem, st>>>(
-        static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
-        static_cast<const T*>(dO), LSE, Dd, n_pad, dQacc, static_cast<T*>(dK),
-        static_cast<T*>(dV), n, m, d, dv, causal, scale);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_BWD_SIMT, st, [&] {
+        kern<<<grid, attn::simt::kThreads, smem, st>>>(
+            static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
+            static_cast<const T*>(dO), LSE, Dd, n_pad, dQacc, static_cast<T*>(dK),
+            static_cast<T*>(dV), n, m, d, dv, causal, scale);
+        return launched();
+    });
 }
 
 template <int D>
@@ -212,10 +265,13 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
         cudaSuccess)
         return ATTN_ERR_CUDA;
     const long long grid = static_cast<long long>((m + kTile - 1) / kTile) * BH;
-    kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-        mq, mk, mv, mdo, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
-        static_cast<__nv_bfloat16*>(dV), n, m, BH, causal, scale, scale * kLog2e, kWaitBudgetNs);
-    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
+        kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
+            mq, mk, mv, mdo, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
+            static_cast<__nv_bfloat16*>(dV), n, m, BH, causal, scale, scale * kLog2e,
+            kWaitBudgetNs);
+        return launched();
+    });
 }
 
 __global__ void probe_timeout_kernel(unsigned long long budget_ns) {
@@ -322,6 +378,34 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     }
     if (s == ATTN_OK) g_last_launches = 3;
     return s;
+}
+
+attn_status_t attn_trace_begin(int capacity) {
+    if (capacity < 1 || capacity > 65536) return ATTN_ERR_SHAPE;
+    g_trace.on = true;
+    g_trace.capacity = capacity;
+    g_trace.entries.clear();
+    return ATTN_OK;
+}
+
+int attn_trace_end(attn_kernel_time_t* out, int max_entries) {
+    TraceState& t = g_trace;
+    t.on = false;
+    const int count = static_cast<int>(t.entries.size());
+    int status = count;
+    for (int k = 0; k < count; ++k) {
+        const TraceEntry& e = t.entries[k];
+        float ms = 0.f;
+        if (cudaEventSynchronize(e.stop) != cudaSuccess ||
+            cudaEventElapsedTime(&ms, e.start, e.stop) != cudaSuccess)
+            status = -1;
+        if (out && k < max_entries) {
+            out[k].kernel = e.kernel;
+            out[k].ms = ms;
+        }
+    }
+    t.entries.clear();
+    return status;
 }
 
 attn_status_t attn_get_device_error(void* stream) {

@@ -267,20 +267,6 @@ def test_matches_torch_autograd_float64(B, H, n, m, d, dv, causal, scale, seed):
         assert rel_to_max(a, b) < 1e-12
 
 
-def test_sampled_rows_match_autograd():
-    rng = np.random.default_rng(9)
-    n = m = 50
-    Q, K, V, dO = (rng.standard_normal((n, 8)) for _ in range(4))
-    q_rows = [0, 7, 31, 49]
-    k_rows = [0, 1, 25, 49]
-    O_s, lse_s, dQ_s, dK_s, dV_s = ref.head_backward_sampled(
-        Q, K, V, dO, q_rows, k_rows, causal=True, row_block=16)
-    tO, tlse, tdQ, tdK, tdV = _torch_ref(Q, K, V, dO, True, None)
-    for a, b in ((O_s, tO[q_rows]), (lse_s, tlse[q_rows]), (dQ_s, tdQ[q_rows]),
-                 (dK_s, tdK[k_rows]), (dV_s, tdV[k_rows])):
-        assert rel_to_max(a, b) < 1e-12
-
-
 def test_row_block_does_not_change_results():
     rng = np.random.default_rng(5)
     Q, K, V, dO = (rng.standard_normal((37, 6)) for _ in range(4))
