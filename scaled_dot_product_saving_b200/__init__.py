@@ -5,7 +5,8 @@ CUDA tensors of one element type, allocates outputs with torch when the caller
 did not pass them, and calls the C entry point of the same name on torch's
 current stream. Every arithmetic step runs in the library's CUDA kernels;
 there is no fallback, and importing this package fails loudly when the
-library has not been built (``python -m scaled_dot_product_saving_b200.build``).
+library has not been built, or is older than the header it must export
+(``python scaled_dot_product_saving_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -44,12 +45,20 @@ class AttnError(RuntimeError):
         super().__init__(f"{where}: {attn_status_string(code)} (status {code})")
 
 
+_BUILD_HINT = "build it with `python scaled_dot_product_saving_b200/build.py` (nvcc, sm_100a)"
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"{LIB_PATH} is missing: build it with "
-            "`python -m scaled_dot_product_saving_b200.build` (nvcc, sm_100a)")
+        raise ImportError(f"{LIB_PATH} is missing: {_BUILD_HINT}")
     L = ctypes.CDLL(LIB_PATH)
+    try:
+        return _declare(L)
+    except AttributeError as e:
+        raise ImportError(f"{LIB_PATH} is stale ({e}): {_BUILD_HINT}") from None
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
     L.attn_fwd.restype = i
@@ -199,3 +208,4 @@ def attn_trace_end(max_entries: int = 65536):
         raise AttnError(7, "attn_trace_end")
     return [(KERNEL_NAMES.get(buf[k].kernel, str(buf[k].kernel)), float(buf[k].ms))
             for k in range(min(count, max_entries))]
+

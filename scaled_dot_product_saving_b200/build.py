@@ -1,6 +1,7 @@
 """Build the in-tree shared library ``libattn.so`` with nvcc for sm_100a.
 
-Usage: ``python -m scaled_dot_product_saving_b200.build [--verbose]``.
+Usage: ``python scaled_dot_product_saving_b200/build.py [--verbose]``. Run it
+by path: importing the package loads the library, which this script builds.
 The library is written next to this file so that it travels with the source
 tree; nothing is installed into site-packages.
 """

@@ -13,8 +13,8 @@ HEADER = os.path.join(ROOT, "include", "attn.h")
 
 @pytest.fixture(scope="module")
 def L():
-    from scaled_dot_product_saving_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import scaled_dot_product_saving_b200 as m
     return m
 
