@@ -107,6 +107,37 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V,
                        attn_dtype_t dtype, int causal, float scale, void* stream);
 
 /*
+ * attn_bwd_noalloc -- attn_bwd for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment convenience, not part
+ * of the method. Some callers cannot hand attn_bwd a workspace: a plugin or
+ * custom op inside a host framework that owns all device memory and gives
+ * the op no scratch buffer, where a cudaMalloc of its own would fail against,
+ * or bypass, the framework's budget. This call takes the same arguments as
+ * attn_bwd minus the workspace, and uses instead a scratch array compiled
+ * into the library: attn_bwd_noalloc_scratch_bytes() bytes (32 MiB) of
+ * device memory that every GPU loading the library holds until the process
+ * exits. It allocates nothing and calls no allocating routine.
+ *  - Sizes whose attn_bwd_workspace_size() exceeds the array are rejected
+ *    with ATTN_ERR_WORKSPACE before anything is launched (the d = 64,
+ *    B*H*n = 65536 problem fits; the long-context ones do not).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture on the device.
+ *  - Every call shares the one array, which keeps the last call's contents;
+ *    the kernels rewrite what they read. Calls whose kernels overlap on the
+ *    GPU (two streams, or two host threads) race on the array: serialise them.
+ * Other statuses are those of attn_bwd.
+ */
+attn_status_t attn_bwd_noalloc(const void* Q, const void* K, const void* V,
+                               const void* O, const void* dO, const float* LSE,
+                               void* dQ, void* dK, void* dV,
+                               int B, int H, int n, int m, int d, int dv,
+                               attn_dtype_t dtype, int causal, float scale, void* stream);
+
+/* Size in bytes of the scratch array attn_bwd_noalloc uses. */
+size_t attn_bwd_noalloc_scratch_bytes(void);
+
+/*
  * attn_get_device_error -- synchronise `stream`, then report and clear the
  * device-side error word of the current device. Every wait inside the
  * tensor-core kernels is bounded; a wait that runs out writes

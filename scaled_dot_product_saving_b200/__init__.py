@@ -22,6 +22,7 @@ __all__ = [
     "attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_error",
     "attn_probe_timeout", "attn_set_path", "attn_last_launch_count", "attn_status_string",
     "dtype_code", "attn_trace_begin", "attn_trace_end", "KERNEL_NAMES",
+    "attn_bwd_noalloc", "attn_bwd_noalloc_scratch_bytes",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
@@ -81,6 +82,11 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.attn_trace_begin.restype = i
     L.attn_trace_end.argtypes = [ctypes.POINTER(_KernelTime), i]
     L.attn_trace_end.restype = i
+    L.attn_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   i, i, i, i, i, i, i, i, f, vp]
+    L.attn_bwd_noalloc.restype = i
+    L.attn_bwd_noalloc_scratch_bytes.argtypes = []
+    L.attn_bwd_noalloc_scratch_bytes.restype = sz
     return L
 
 
@@ -209,3 +215,21 @@ def attn_trace_end(max_entries: int = 65536):
     return [(KERNEL_NAMES.get(buf[k].kernel, str(buf[k].kernel)), float(buf[k].ms))
             for k in range(min(count, max_entries))]
 
+
+def attn_bwd_noalloc_scratch_bytes() -> int:
+    return int(lib.attn_bwd_noalloc_scratch_bytes())
+
+
+def attn_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal=False, scale=None, stream=None):
+    """attn_bwd without a workspace: the library's own fixed scratch array is
+    used, for callers that may not allocate device memory. The caller still
+    passes every input and output tensor; nothing is allocated here."""
+    _require(q, k, v, o, do, dq, dk, dv)
+    B, H, n, m, d, dvw = _dims(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    _check(lib.attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, H, n, m, d, dvw,
+                                dtype_code(q.dtype), int(bool(causal)), scale,
+                                _stream_handle(stream)),
+           "attn_bwd_noalloc")
+    return dq, dk, dv

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libattn.so")
-SOURCES = [os.path.join(CSRC, "attn.cu")]
+SOURCES = [os.path.join(CSRC, "attn.cu"), os.path.join(CSRC, "noalloc.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] \
     + [os.path.join(INCLUDE, "attn.h")]
 
