@@ -172,13 +172,16 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- multi-rank
-def init_distributed():
+def init_distributed(backend=None):
+    """Join the process group described by RANK / WORLD_SIZE / LOCAL_RANK
+    (torch.distributed.run sets them); NCCL on GPUs, gloo otherwise."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
