@@ -92,21 +92,29 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [BH, rows, width] bf16 viewed as 3-D (width innermost); boxes of 64 x 128 x 1
-// with the 128-byte swizzle the UMMA descriptors expect.
-bool make_map(CUtensorMap* map, const void* base, int width, int rows, int bh) {
+// [BH, rows, width] viewed as 3-D (width innermost) with the 128-byte swizzle.
+// bf16 operand tiles use boxes of 64 x 128 x 1 (the layout the UMMA
+// descriptors expect); the fp32 dQ accumulator uses 32 x 32 x 1 boxes for the
+// dQ warpgroup's reduce-adds.
+bool make_map_typed(CUtensorMap* map, const void* base, int width, int rows, int bh,
+                    CUtensorMapDataType type, int elem_bytes, int box_x, int box_y) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(bh)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(width) * 2,
-                             static_cast<cuuint64_t>(width) * 2 * rows};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTile), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(width) * elem_bytes,
+                             static_cast<cuuint64_t>(width) * elem_bytes * rows};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return enc(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int width, int rows, int bh) {
+    return make_map_typed(map, base, width, rows, bh, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64,
+                          kTile);
 }
 
 // ---------------------------------------------------------------- tracing
@@ -195,7 +203,8 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
 
 template <typename T>
 attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float* lse2, float* Dd,
-                         float* dQacc, int BH, int n, int n_pad, int d, int dv, cudaStream_t st) {
+                         float* dQacc, int BH, int n, int n_pad, int d, int dv, float d_scale,
+                         cudaStream_t st) {
     const size_t rows = static_cast<size_t>(BH) * n_pad;
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
     const bool vec = sizeof(T) == 2 && dv % 8 == 0 && (dv / 8) <= 32 && 32 % (dv / 8) == 0 &&
@@ -206,7 +215,7 @@ attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float*
         return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
             attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
-                lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv);
+                lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv, d_scale);
             return launched();
         });
     }
@@ -214,7 +223,7 @@ attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float*
     return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
         attn::prep::preprocess_generic<T><<<grid, attn::prep::kThreads, 0, st>>>(
             static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, dq_elems,
-            BH, n, n_pad, dv);
+            BH, n, n_pad, dv, d_scale);
         return launched();
     });
 }
@@ -256,9 +265,10 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
                          void* dV, int BH, int n, int m, int causal, float scale,
                          cudaStream_t st) {
     using C = attn::bwdtc::Cfg<D>;
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mdq;
     if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) ||
-        !make_map(&mv, V, D, m, BH) || !make_map(&mdo, dO, D, n, BH))
+        !make_map(&mv, V, D, m, BH) || !make_map(&mdo, dO, D, n, BH) ||
+        !make_map_typed(&mdq, dQacc, D, n, BH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 32, 32))
         return ATTN_ERR_CUDA;
     auto kern = attn::bwdtc::bwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
@@ -267,7 +277,7 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     const long long grid = static_cast<long long>((m + kTile - 1) / kTile) * BH;
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mdo, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
+            mq, mk, mv, mdo, mdq, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
             static_cast<__nv_bfloat16*>(dV), n, m, BH, causal, scale, scale * kLog2e,
             kWaitBudgetNs);
         return launched();
@@ -357,9 +367,12 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     float* dQacc = reinterpret_cast<float*>(ws + w.dq_off);
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
 
+    // The tensor-core backward takes D already multiplied by the scale.
+    const float d_scale = tensor ? scale : 1.0f;
     s = (dtype == ATTN_F32)
-            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, st)
-            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, st);
+            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, d_scale, st)
+            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv,
+                                        d_scale, st);
     if (s != ATTN_OK) return s;
     if (tensor) {
         s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, w.n_pad, dQacc, dK, dV, BH, n, m,

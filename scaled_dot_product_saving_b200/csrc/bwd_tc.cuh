@@ -6,16 +6,25 @@
 //   S^T  = K_j Q_i^T                  tcgen05 (A = K_j, B = Q_i, both K-major)
 //   dP^T = V_j dO_i^T                 tcgen05 (A = V_j, B = dO_i)
 //   P^T  = 2^(S^T*scale*log2e - LSE_i*log2e), 0 where masked
-//   dS^T = scale * P^T * (dP^T - D_i)            (128 threads, one key each)
+//   dS^T = P^T * (scale*dP^T - scale*D_i)        (128 threads, one key each)
 //   dV_j += P^T dO_i                  tcgen05, A = P^T from TMEM (bf16 written
 //                                     over its own S^T columns), B = dO_i MN-major
 //   dK_j += dS^T Q_i                  tcgen05, A = dS^T from TMEM, B = Q_i MN-major
 //   dQ_i += dS K_j                    tcgen05, A = dS from shared memory
-//                                     (MN-major), B = K_j (MN-major); the fp32
-//                                     result is reduce-added into the global dQ
-//                                     accumulator by a second warpgroup.
+//                                     (MN-major), B = K_j (MN-major); a second
+//                                     warpgroup stages the fp32 result through
+//                                     the (by then free) dS tile and hands it to
+//                                     the TMA engine as tiled reduce-adds into
+//                                     the global dQ accumulator.
 // dV_j and dK_j stay in TMEM across all query tiles and are written once.
 // Folding `scale` into dS makes dK and dQ come out already scaled.
+//
+// The P/dS warpgroup works through a tile in four chunks of 32 queries and
+// signals each chunk as soon as its P^T/dS^T are in TMEM, so the MMA thread
+// issues that chunk's dV/dK k-steps while the warpgroup computes the next
+// chunk. CTAs are ordered head-major, so the key tiles of one head run
+// together and share its Q/dO tiles and its slice of the dQ accumulator
+// through L2.
 //
 // Where the pages stand: dV, dP, dS, dQ and dK are "Attention Backward Pass
 // (dQ, dK, dV)", section "Backward", and "Attention backward", Problems 2-6;
@@ -29,10 +38,12 @@
 // warpgroup (TMEM lane = query row).
 //
 // TMEM (512 columns). d = 128: dV [0,128) dK [128,256) S^T [256,384)
-// dP^T [384,512); P^T (bf16) goes to [256,320), dS^T to [384,448), and the two
-// 64-column halves of dQ to [320,384) and [448,512) -- columns whose fp32
-// contents have been consumed by then. d = 64: dV [0,64) dK [64,128)
-// S^T [128,256) dP^T [256,384) dQ [384,448).
+// dP^T [384,512); P^T (bf16) goes to [256,320) and dS^T to [384,448); dQ then
+// takes all of [256,384). The tensor pipe runs MMAs in issue order, so the dQ
+// MMA, issued after the last dV MMA, overwrites P^T only once it has been
+// read; the next tile's dP^T MMA is issued before the dQ drain is awaited and
+// only its S^T MMA waits for it. d = 64: dV [0,64) dK [64,128) S^T [128,256)
+// dP^T [256,384) dQ [384,448).
 #pragma once
 
 #include "sm100.cuh"
@@ -42,6 +53,7 @@ namespace bwdtc {
 
 constexpr int kBN = 128;      // keys per CTA
 constexpr int kBM = 128;      // queries per tile
+constexpr int kChunks = 4;    // 32-query chunks of a tile
 constexpr int kThreads = 384;
 
 template <int D>
@@ -67,8 +79,11 @@ struct Cfg {
     static constexpr uint32_t kColdP = 2 * D + 128;
     static constexpr uint32_t kColP = kColS;          // bf16 P^T over S^T
     static constexpr uint32_t kColdS = kColdP;        // bf16 dS^T over dP^T
-    static constexpr uint32_t kColdQ0 = kAlias ? kColS + 64 : 2 * D + 256;
-    static constexpr uint32_t kColdQ1 = kAlias ? kColdP + 64 : kColdQ0 + 64;
+    static constexpr uint32_t kColdQ = kAlias ? kColS : 2 * D + 256;
+    // dQ staging through the dS tile: per warp, two 32-row x 32-column fp32
+    // buffers (4 KB each, 128B-swizzled) that alternate over the row's D/32
+    // segments.
+    static constexpr int kStageWarpBytes = 8192;
 };
 
 struct Bars {
@@ -76,20 +91,61 @@ struct Bars {
     uint64_t q_full[4];
     uint64_t q_empty[4];
     uint64_t s_full;
-    uint64_t ds_full;
+    uint64_t ds_chunk[kChunks];
     uint64_t dq_full;
     uint64_t dq_free;
+    uint64_t ds_smem_free;
     uint64_t acc_done;
     uint64_t mma_drain;
     uint32_t tmem_base;
     int abort;
 };
 
+// One 32-query chunk of the P/dS warpgroup: P^T and dS^T from the S^T / dP^T
+// values in registers, written back to TMEM and (dS) to shared memory.
+template <int D>
+__device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const uint32_t (&pr)[32],
+                                          const float* lse_s, const float* dd_s, bool masked,
+                                          int r, int keys_masked_below, float scale,
+                                          float scale_log2, uint32_t tmem_lane, uint8_t* sdS) {
+    using C = Cfg<D>;
+    uint32_t pk[16], dk[16];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + 4 * g);
+        const float4 d4 = *reinterpret_cast<const float4*>(dd_s + c * 32 + 4 * g);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+        float p[4], ds[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int e = 4 * g + h;
+            p[h] = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, -lv[h]));
+            if (masked && (c * 32 + e) < keys_masked_below) p[h] = 0.f;
+            ds[h] = p[h] * fmaf(__uint_as_float(pr[e]), scale, -dv[h]);
+        }
+        pk[2 * g] = pack_bf16x2(p[0], p[1]);
+        pk[2 * g + 1] = pack_bf16x2(p[2], p[3]);
+        dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
+        dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
+    }
+    tmem_st16(tmem_lane + C::kColP + c * 16, pk);
+    tmem_st16(tmem_lane + C::kColdS + c * 16, dk);
+    // dS (queries contiguous, 128B-swizzled) for the dQ MMA's A operand.
+    uint8_t* rowp = sdS + (c >> 1) * C::kPanelBytes + r * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int chunk = ((c & 1) * 4 + q) ^ (r & 7);
+        *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+            make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-           const float* __restrict__ lse2, const float* __restrict__ Dd, int n_pad,
+           const __grid_constant__ CUtensorMap tmdQacc, const float* __restrict__ lse2, const float* __restrict__ Dd, int n_pad,
            float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dK,
            __nv_bfloat16* __restrict__ dV, int n, int m, int BH, int causal, float scale,
            float scale_log2, unsigned long long budget_ns) {
@@ -99,8 +155,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int kt = int(blockIdx.x / BH);      // key tile; low tiles (most work if causal) first
-    const int bh = int(blockIdx.x % BH);
+    const int num_kt = (m + kBN - 1) / kBN;
+    const int bh = int(blockIdx.x / num_kt);  // head-major: one head's key tiles together,
+    const int kt = int(blockIdx.x % num_kt);  // the longest (lowest, if causal) first
     const int k0 = kt * kBN;
     const int num_qt = (n + kBM - 1) / kBM;
     const int first_qt = causal ? kt : 0;
@@ -118,9 +175,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mbar_init(&bars->q_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->ds_full, 128);
+        for (int c = 0; c < kChunks; ++c) mbar_init(&bars->ds_chunk[c], 128);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_free, 128);
+        mbar_init(&bars->ds_smem_free, 128);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->mma_drain, 1);
         fence_mbar_init();
@@ -141,6 +199,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         prefetch_tensor_map(&tmK);
         prefetch_tensor_map(&tmV);
         prefetch_tensor_map(&tmdO);
+        prefetch_tensor_map(&tmdQacc);
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p) {
             tma_load_3d(smem + C::kOffK + p * C::kPanelBytes, &tmK, &bars->kv_full, p * 64, k0, bh);
@@ -176,7 +235,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
-        constexpr uint32_t idQ = idesc_bf16_f32(kBM, 64, 1, 1);     // dQ, one 64-wide half
+        constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 1, 1);      // dQ
         const uint32_t sK = smem_addr(smem + C::kOffK);
         const uint32_t sV = smem_addr(smem + C::kOffV);
         const uint32_t sdS = smem_addr(smem + C::kOffdS);
@@ -189,6 +248,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 ok = false;
                 break;
             }
+            tc_fence_after();
+            // dP^T first: its columns are free once the previous dK MMAs
+            // (issued earlier) have read dS^T from them.
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
+            }
+            // S^T shares its columns with the previous tile's dQ (d = 128).
             if (C::kAlias && t > 0 &&
                 !mbar_wait(&bars->dq_free, (t - 1) & 1, abort_flag, budget_ns)) {
                 ok = false;
@@ -201,26 +270,27 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
                        sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
             }
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
-            }
             mma_commit(&bars->s_full);
-            if (!mbar_wait(&bars->ds_full, t & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
+            // dV += P^T dO and dK += dS^T Q, 32 queries (two k-steps) per chunk
+            // as soon as the P/dS warpgroup has written that chunk.
+            for (int c = 0; c < kChunks; ++c) {
+                if (!mbar_wait(&bars->ds_chunk[c], t & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
+                    mma_ts(tmem + C::kColdV, tmem + C::kColP + kk * 8,
+                           sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV,
+                           (t > 0 || kk > 0));
+#pragma unroll
+                for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
+                    mma_ts(tmem + C::kColdK, tmem + C::kColdS + kk * 8,
+                           sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV,
+                           (t > 0 || kk > 0));
             }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kBM / 16; ++kk)
-                mma_ts(tmem + C::kColdV, tmem + C::kColP + kk * 8,
-                       sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, (t > 0 || kk > 0));
-#pragma unroll
-            for (int kk = 0; kk < kBM / 16; ++kk)
-                mma_ts(tmem + C::kColdK, tmem + C::kColdS + kk * 8,
-                       sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, (t > 0 || kk > 0));
+            if (!ok) break;
             mma_commit(&bars->q_empty[s]);
             if (t == T - 1) mma_commit(&bars->acc_done);
             if (!C::kAlias && t > 0 &&
@@ -228,15 +298,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 ok = false;
                 break;
             }
+            tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < C::kPanels; ++h) {
-                const uint32_t dq = tmem + (h == 0 ? C::kColdQ0 : C::kColdQ1);
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ss(dq, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
-                           sdesc_sw128(sK + h * C::kPanelBytes + kk * 2048, C::kPanelBytes, 1024),
-                           idQ, kk > 0);
-            }
+            for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ss(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
+                       sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0);
             mma_commit(&bars->dq_full);
         }
         if (!ok) {
@@ -248,7 +314,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     } else if (!aborted_early && warp >= 4 && warp < 8) {
         // ------------------------------------------------ P / dS warpgroup
         const int r = threadIdx.x - 128;                 // key row in the tile == TMEM lane
-        const uint32_t lane_sel = uint32_t((warp & 3) * 32) << 16;
+        const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16);
         const int j = k0 + r;
         const bool key_ok = j < m;
         uint8_t* sdS = smem + C::kOffdS;
@@ -256,51 +322,50 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int t = 0; t < T; ++t) {
             const int s = t % C::kStages;
             const int q0 = (first_qt + t) * kBM;
+            // The dS tile is also the dQ warpgroup's staging buffer for the
+            // previous tile: wait until the TMA engine has read it.
             if (!mbar_wait_warp(&bars->q_full[s], (t / C::kStages) & 1, abort_flag, budget_ns) ||
-                !mbar_wait_warp(&bars->s_full, t & 1, abort_flag, budget_ns)) {
+                !mbar_wait_warp(&bars->s_full, t & 1, abort_flag, budget_ns) ||
+                (t > 0 &&
+                 !mbar_wait_warp(&bars->ds_smem_free, (t - 1) & 1, abort_flag, budget_ns))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             const float* lse_s = reinterpret_cast<const float*>(smem + C::kOffLse + s * kBM * 4);
             const float* dd_s = reinterpret_cast<const float*>(smem + C::kOffDd + s * kBM * 4);
+            // Keys past the end get P = 0 in every column; on the diagonal tile,
+            // key r is masked for the queries in the tile before it (q < r).
             const bool diag = causal && (q0 == k0);
+            const bool masked = !key_ok || diag;
+            const int below = key_ok ? r : kBM;
+            // Chunk c's TMEM loads are issued while chunk c-1 is processed.
+            uint32_t s0[32], p0[32], s1[32], p1[32];
+            tmem_ld32(tl + C::kColS, s0);
+            tmem_ld32(tl + C::kColdP, p0);
+            tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < kBM / 32; ++c) {
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tmem + lane_sel + C::kColS + c * 32, sr);
-                tmem_ld32(tmem + lane_sel + C::kColdP + c * 32, pr);
+            for (int c = 0; c < kChunks; c += 2) {
+                tmem_ld32(tl + C::kColS + (c + 1) * 32, s1);
+                tmem_ld32(tl + C::kColdP + (c + 1) * 32, p1);
+                pds_chunk<D>(c, s0, p0, lse_s, dd_s, masked, r, below, scale, scale_log2, tl, sdS);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars->ds_chunk[c]);
                 tmem_ld_wait();
-                uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float pp[2], dd[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int qi = c * 32 + 2 * e + h;
-                        float p = ex2(fmaf(__uint_as_float(sr[2 * e + h]), scale_log2, -lse_s[qi]));
-                        if (!key_ok || (diag && qi < r)) p = 0.f;
-                        pp[h] = p;
-                        dd[h] = p * (__uint_as_float(pr[2 * e + h]) - dd_s[qi]) * scale;
-                    }
-                    pk[e] = pack_bf16x2(pp[0], pp[1]);
-                    dk[e] = pack_bf16x2(dd[0], dd[1]);
+                if (c + 2 < kChunks) {
+                    tmem_ld32(tl + C::kColS + (c + 2) * 32, s0);
+                    tmem_ld32(tl + C::kColdP + (c + 2) * 32, p0);
                 }
-                tmem_st16(tmem + lane_sel + C::kColP + c * 16, pk);
-                tmem_st16(tmem + lane_sel + C::kColdS + c * 16, dk);
-                // dS (queries contiguous, 128B-swizzled) for the dQ MMA's A operand.
-                uint8_t* rowp = sdS + (c >> 1) * C::kPanelBytes + r * 128;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = ((c & 1) * 4 + q) ^ (r & 7);
-                    *reinterpret_cast<uint4*>(rowp + chunk * 16) =
-                        make_uint4(dk[4 * q], dk[4 * q + 1], dk[4 * q + 2], dk[4 * q + 3]);
-                }
+                pds_chunk<D>(c + 1, s1, p1, lse_s, dd_s, masked, r, below, scale, scale_log2, tl,
+                             sdS);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bars->ds_chunk[c + 1]);
+                if (c + 2 < kChunks) tmem_ld_wait();
             }
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars->ds_full);
         }
         if (ok && !mbar_wait_warp(&bars->acc_done, 0, abort_flag, budget_ns)) ok = false;
         if (ok) {
@@ -314,7 +379,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t rr[32];
-                    tmem_ld32(tmem + lane_sel + col + c * 32, rr);
+                    tmem_ld32(tl + col + c * 32, rr);
                     tmem_ld_wait();
                     if (key_ok) {
 #pragma unroll
@@ -335,11 +400,19 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
     } else if (!aborted_early && warp >= 8) {
         // ------------------------------------------------ dQ warpgroup
-        const int r = threadIdx.x - 256;                 // query row in the tile == TMEM lane
-        const uint32_t lane_sel = uint32_t((warp & 3) * 32) << 16;
+        // Thread r owns query row r of the tile (its TMEM lane). Once the dQ
+        // MMA has completed, the dS tile is free until the P/dS warpgroup
+        // writes the next tile's dS. Each warp stages its 32 rows there one
+        // 32-column segment at a time, in the 128-byte swizzled layout of the
+        // accumulator's tensor map, and one lane hands each segment to the
+        // TMA engine as a tiled reduce-add; rows past n are clipped by the TMA.
+        const int r = threadIdx.x - 256;
+        const int wq = warp & 3;
+        const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
+        uint8_t* stage = smem + C::kOffdS + wq * C::kStageWarpBytes;
         bool ok = true;
         for (int t = 0; t < T; ++t) {
-            const int i = (first_qt + t) * kBM + r;
+            const int row0 = (first_qt + t) * kBM + wq * 32;
             if (!mbar_wait_warp(&bars->dq_full, t & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
@@ -347,23 +420,36 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tc_fence_after();
             uint32_t v[D];
 #pragma unroll
-            for (int h = 0; h < C::kPanels; ++h) {
-                const uint32_t col = h == 0 ? C::kColdQ0 : C::kColdQ1;
-                tmem_ld32(tmem + lane_sel + col, *reinterpret_cast<uint32_t(*)[32]>(v + 64 * h));
-                tmem_ld32(tmem + lane_sel + col + 32,
-                          *reinterpret_cast<uint32_t(*)[32]>(v + 64 * h + 32));
-            }
+            for (int c = 0; c < D / 32; ++c)
+                tmem_ld32(tl + C::kColdQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&bars->dq_free);
-            if (i < n) {
-                float* dst = dQacc + (size_t(bh) * n + i) * D;
 #pragma unroll
-                for (int c = 0; c < D; c += 4)
-                    red_add_v4(dst + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                               __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+            for (int g = 0; g < D / 32; ++g) {
+                uint8_t* buf = stage + (g & 1) * 4096;
+                if (g >= 2) {
+                    if (lane == 0) bulk_wait_group_read1();   // buffer g-2 read
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                        make_uint4(v[32 * g + 4 * k], v[32 * g + 4 * k + 1], v[32 * g + 4 * k + 2],
+                                   v[32 * g + 4 * k + 3]);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_reduce_add_3d(&tmdQacc, buf, 32 * g, row0, bh);
+                    bulk_commit_group();
+                }
             }
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+            mbar_arrive(&bars->ds_smem_free);
         }
+        if (lane == 0) bulk_wait_group0();
+        __syncwarp();
         if (!ok) {
             record_device_error(kErrTimeout);
             *abort_flag = 1;

@@ -5,7 +5,8 @@
 //   O(n dv) instead of O(n m). It also writes the forward's LSE in base 2,
 //   and both arrays are padded to whole 128-row tiles (D = 0 and LSE = +inf
 //   in the padding, so padded query rows get P = 0 on the tensor-core path).
-//   The same launch zeroes the fp32 dQ accumulator.
+//   The same launch zeroes the fp32 dQ accumulator. D is stored multiplied by
+//   `d_scale` (the tensor-core backward folds the attention scale into it).
 // finalize: dQ = post_scale * dQacc, converted to the element type.
 #pragma once
 
@@ -40,7 +41,7 @@ __global__ void __launch_bounds__(kThreads)
 preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                     const float* __restrict__ LSE, float* __restrict__ lse2,
                     float* __restrict__ Dd, float* __restrict__ dQacc, size_t dq_elems,
-                    int BH, int n, int n_pad, int dv) {
+                    int BH, int n, int n_pad, int dv, float d_scale) {
     const int G = dv / 8;                       // lanes per row
     const int rows_per_warp = 32 / G;
     const int lane = threadIdx.x & 31;
@@ -63,7 +64,7 @@ preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __
         }
         for (int off = G / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (row < total_rows && lig == 0) {
-            Dd[row] = real ? s : 0.f;
+            Dd[row] = real ? s * d_scale : 0.f;
             lse2[row] = real ? LSE[src] * kLog2e : INFINITY;
         }
     }
@@ -84,7 +85,7 @@ __global__ void __launch_bounds__(kThreads)
 preprocess_generic(const T* __restrict__ O, const T* __restrict__ dO,
                    const float* __restrict__ LSE, float* __restrict__ lse2,
                    float* __restrict__ Dd, float* __restrict__ dQacc, size_t dq_elems, int BH,
-                   int n, int n_pad, int dv) {
+                   int n, int n_pad, int dv, float d_scale) {
     const int lane = threadIdx.x & 31;
     const size_t warp_global = (size_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const size_t nwarps = (size_t(gridDim.x) * kThreads) >> 5;
@@ -98,7 +99,7 @@ preprocess_generic(const T* __restrict__ O, const T* __restrict__ dO,
             for (int c = lane; c < dv; c += 32) s = fmaf(ld_f(O + src * dv + c), ld_f(dO + src * dv + c), s);
         for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
         if (lane == 0) {
-            Dd[row] = (i < n) ? s : 0.f;
+            Dd[row] = (i < n) ? s * d_scale : 0.f;
             lse2[row] = (i < n) ? LSE[src] * kLog2e : INFINITY;
         }
     }
