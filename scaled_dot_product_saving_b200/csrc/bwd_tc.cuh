@@ -19,12 +19,17 @@
 // dV_j and dK_j stay in TMEM across all query tiles and are written once.
 // Folding `scale` into dS makes dK and dQ come out already scaled.
 //
-// The P/dS warpgroup works through a tile in four chunks of 32 queries and
-// signals each chunk as soon as its P^T/dS^T are in TMEM, so the MMA thread
-// issues that chunk's dV/dK k-steps while the warpgroup computes the next
-// chunk. CTAs are ordered head-major, so the key tiles of one head run
-// together and share its Q/dO tiles and its slice of the dQ accumulator
-// through L2.
+// Two P/dS warpgroups split a tile into four chunks of 32 queries (two chunks
+// each) and signal each chunk as soon as its P^T/dS^T are in TMEM, so the MMA
+// thread issues that chunk's dV/dK k-steps while the chunks after it are
+// computed; with two warps per SM sub-partition each hides the other's
+// latencies. Each chunk's P^T/dS^T go into the first 16 of its own 32 TMEM
+// columns, so no chunk overwrites data another chunk has yet to read. dS for
+// the dQ MMA is kept in registers and written to shared memory only at the
+// end of the tile, by when the dQ warpgroup has normally finished staging the
+// previous tile's dQ through that buffer. CTAs are ordered head-major, so the
+// key tiles of one head run together and share its Q/dO tiles and its slice
+// of the dQ accumulator through L2.
 //
 // Where the pages stand: dV, dP, dS, dQ and dK are "Attention Backward Pass
 // (dQ, dK, dV)", section "Backward", and "Attention backward", Problems 2-6;
@@ -33,13 +38,13 @@
 // exact zeros ("Attention backward", Problem 8), so tiles wholly above the
 // diagonal are skipped.
 //
-// Warp roles (384 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// MMA issuer, warps 4-7 = P/dS warpgroup (TMEM lane = key), warps 8-11 = dQ
-// warpgroup (TMEM lane = query row).
+// Warp roles (448 threads): warps 0-3 and 4-7 = the two P/dS warpgroups (TMEM
+// lane = key), warps 8-11 = dQ warpgroup (TMEM lane = query row), warp 12 =
+// TMA producer, warp 13 = TMEM allocator and MMA issuer.
 //
 // TMEM (512 columns). d = 128: dV [0,128) dK [128,256) S^T [256,384)
-// dP^T [384,512); P^T (bf16) goes to [256,320) and dS^T to [384,448); dQ then
-// takes all of [256,384). The tensor pipe runs MMAs in issue order, so the dQ
+// dP^T [384,512); chunk c's P^T (bf16) goes to [256+32c, 256+32c+16) and its
+// dS^T to [384+32c, 384+32c+16); dQ then takes all of [256,384). The tensor pipe runs MMAs in issue order, so the dQ
 // MMA, issued after the last dV MMA, overwrites P^T only once it has been
 // read; the next tile's dP^T MMA is issued before the dQ drain is awaited and
 // only its S^T MMA waits for it. d = 64: dV [0,64) dK [64,128) S^T [128,256)
@@ -54,7 +59,10 @@ namespace bwdtc {
 constexpr int kBN = 128;      // keys per CTA
 constexpr int kBM = 128;      // queries per tile
 constexpr int kChunks = 4;    // 32-query chunks of a tile
-constexpr int kThreads = 384;
+constexpr int kThreads = 448;
+constexpr int kWarpDq = 8;         // first warp of the dQ warpgroup
+constexpr int kWarpProducer = 12;
+constexpr int kWarpMma = 13;
 
 template <int D>
 struct Cfg {
@@ -94,6 +102,7 @@ struct Bars {
     uint64_t ds_chunk[kChunks];
     uint64_t dq_full;
     uint64_t dq_free;
+    uint64_t ds_smem_full;
     uint64_t ds_smem_free;
     uint64_t acc_done;
     uint64_t mma_drain;
@@ -101,15 +110,17 @@ struct Bars {
     int abort;
 };
 
-// One 32-query chunk of the P/dS warpgroup: P^T and dS^T from the S^T / dP^T
-// values in registers, written back to TMEM and (dS) to shared memory.
+// One 32-query chunk c of a P/dS warpgroup: P^T and dS^T from the S^T / dP^T
+// values in registers, written back to TMEM over the first 16 of the chunk's
+// own 32 S^T / dP^T columns; the packed dS is returned in `dk` for the shared
+// memory tile.
 template <int D>
 __device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const uint32_t (&pr)[32],
                                           const float* lse_s, const float* dd_s, bool masked,
-                                          int r, int keys_masked_below, float scale,
-                                          float scale_log2, uint32_t tmem_lane, uint8_t* sdS) {
+                                          int keys_masked_below, float scale, float scale_log2,
+                                          uint32_t tmem_lane, uint32_t (&dk)[16]) {
     using C = Cfg<D>;
-    uint32_t pk[16], dk[16];
+    uint32_t pk[16];
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + 4 * g);
@@ -129,9 +140,15 @@ __device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const
         dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
         dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
     }
-    tmem_st16(tmem_lane + C::kColP + c * 16, pk);
-    tmem_st16(tmem_lane + C::kColdS + c * 16, dk);
-    // dS (queries contiguous, 128B-swizzled) for the dQ MMA's A operand.
+    tmem_st16(tmem_lane + C::kColP + c * 32, pk);
+    tmem_st16(tmem_lane + C::kColdS + c * 32, dk);
+}
+
+// dS of chunk c for key row r into the shared tile (queries contiguous,
+// 128B-swizzled), the dQ MMA's A operand.
+template <int D>
+__device__ __forceinline__ void store_ds_chunk(uint8_t* sdS, int c, int r, const uint32_t (&dk)[16]) {
+    using C = Cfg<D>;
     uint8_t* rowp = sdS + (c >> 1) * C::kPanelBytes + r * 128;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -178,12 +195,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int c = 0; c < kChunks; ++c) mbar_init(&bars->ds_chunk[c], 128);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_free, 128);
+        mbar_init(&bars->ds_smem_full, 256);
         mbar_init(&bars->ds_smem_free, 128);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->mma_drain, 1);
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(&bars->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
@@ -193,7 +211,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t tmem = bars->tmem_base;
     const bool aborted_early = bars->abort != 0 || T <= 0;
 
-    if (!aborted_early && warp == 0 && lane == 0) {
+    if (!aborted_early && warp == kWarpProducer && lane == 0) {
         // ------------------------------------------------ TMA producer
         prefetch_tensor_map(&tmQ);
         prefetch_tensor_map(&tmK);
@@ -231,7 +249,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         (void)mbar_wait_timed(&bars->kv_full, 0, budget_ns);
         for (int t = (issued > C::kStages ? issued - C::kStages : 0); t < issued; ++t)
             (void)mbar_wait_timed(&bars->q_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == 1 && lane == 0) {
+    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
@@ -272,29 +290,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
             mma_commit(&bars->s_full);
             // dV += P^T dO and dK += dS^T Q, 32 queries (two k-steps) per chunk
-            // as soon as the P/dS warpgroup has written that chunk.
-            for (int c = 0; c < kChunks; ++c) {
+            // as soon as a P/dS warpgroup has written that chunk; the two
+            // warpgroups finish chunks 0 and 2 first, then 1 and 3.
+            bool first = (t == 0);
+            for (int ci = 0; ci < kChunks; ++ci) {
+                const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
                 if (!mbar_wait(&bars->ds_chunk[c], t & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
-                    mma_ts(tmem + C::kColdV, tmem + C::kColP + kk * 8,
-                           sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV,
-                           (t > 0 || kk > 0));
-#pragma unroll
-                for (int kk = 2 * c; kk < 2 * c + 2; ++kk)
-                    mma_ts(tmem + C::kColdK, tmem + C::kColdS + kk * 8,
-                           sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV,
-                           (t > 0 || kk > 0));
+                for (int h = 0; h < 2; ++h) {
+                    const int kk = 2 * c + h;                      // queries 16kk..16kk+15
+                    mma_ts(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
+                           sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                    mma_ts(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
+                           sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                    first = false;
+                }
             }
             if (!ok) break;
             mma_commit(&bars->q_empty[s]);
             if (t == T - 1) mma_commit(&bars->acc_done);
             if (!C::kAlias && t > 0 &&
                 !mbar_wait(&bars->dq_free, (t - 1) & 1, abort_flag, budget_ns)) {
+                ok = false;
+                break;
+            }
+            if (!mbar_wait(&bars->ds_smem_full, t & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
@@ -311,9 +335,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         mma_commit(&bars->mma_drain);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
-    } else if (!aborted_early && warp >= 4 && warp < 8) {
-        // ------------------------------------------------ P / dS warpgroup
-        const int r = threadIdx.x - 128;                 // key row in the tile == TMEM lane
+    } else if (!aborted_early && warp < 8) {
+        // ------------------------------------------------ P / dS warpgroups
+        const int grp = warp >> 2;                       // chunks 2*grp and 2*grp+1
+        const int r = threadIdx.x & 127;                 // key row in the tile == TMEM lane
         const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16);
         const int j = k0 + r;
         const bool key_ok = j < m;
@@ -322,12 +347,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int t = 0; t < T; ++t) {
             const int s = t % C::kStages;
             const int q0 = (first_qt + t) * kBM;
-            // The dS tile is also the dQ warpgroup's staging buffer for the
-            // previous tile: wait until the TMA engine has read it.
             if (!mbar_wait_warp(&bars->q_full[s], (t / C::kStages) & 1, abort_flag, budget_ns) ||
-                !mbar_wait_warp(&bars->s_full, t & 1, abort_flag, budget_ns) ||
-                (t > 0 &&
-                 !mbar_wait_warp(&bars->ds_smem_free, (t - 1) & 1, abort_flag, budget_ns))) {
+                !mbar_wait_warp(&bars->s_full, t & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
@@ -339,33 +360,40 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const bool diag = causal && (q0 == k0);
             const bool masked = !key_ok || diag;
             const int below = key_ok ? r : kBM;
-            // Chunk c's TMEM loads are issued while chunk c-1 is processed.
-            uint32_t s0[32], p0[32], s1[32], p1[32];
-            tmem_ld32(tl + C::kColS, s0);
-            tmem_ld32(tl + C::kColdP, p0);
-            tmem_ld_wait();
-#pragma unroll
-            for (int c = 0; c < kChunks; c += 2) {
-                tmem_ld32(tl + C::kColS + (c + 1) * 32, s1);
-                tmem_ld32(tl + C::kColdP + (c + 1) * 32, p1);
-                pds_chunk<D>(c, s0, p0, lse_s, dd_s, masked, r, below, scale, scale_log2, tl, sdS);
+            uint32_t ds0[16], ds1[16];
+            {
+                const int c = 2 * grp;
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tl + C::kColS + c * 32, sr);
+                tmem_ld32(tl + C::kColdP + c * 32, pr);
+                tmem_ld_wait();
+                pds_chunk<D>(c, sr, pr, lse_s, dd_s, masked, below, scale, scale_log2, tl, ds0);
                 tmem_st_wait();
-                fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bars->ds_chunk[c]);
-                tmem_ld_wait();
-                if (c + 2 < kChunks) {
-                    tmem_ld32(tl + C::kColS + (c + 2) * 32, s0);
-                    tmem_ld32(tl + C::kColdP + (c + 2) * 32, p0);
-                }
-                pds_chunk<D>(c + 1, s1, p1, lse_s, dd_s, masked, r, below, scale, scale_log2, tl,
-                             sdS);
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bars->ds_chunk[c + 1]);
-                if (c + 2 < kChunks) tmem_ld_wait();
             }
+            {
+                const int c = 2 * grp + 1;
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tl + C::kColS + c * 32, sr);
+                tmem_ld32(tl + C::kColdP + c * 32, pr);
+                tmem_ld_wait();
+                pds_chunk<D>(c, sr, pr, lse_s, dd_s, masked, below, scale, scale_log2, tl, ds1);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&bars->ds_chunk[c]);
+            }
+            // The dS tile doubles as the dQ warpgroup's staging buffer for the
+            // previous tile: write it once the TMA engine has read that.
+            if (t > 0 &&
+                !mbar_wait_warp(&bars->ds_smem_free, (t - 1) & 1, abort_flag, budget_ns)) {
+                ok = false;
+                break;
+            }
+            store_ds_chunk<D>(sdS, 2 * grp, r, ds0);
+            store_ds_chunk<D>(sdS, 2 * grp + 1, r, ds1);
+            fence_proxy_async_smem();
+            mbar_arrive(&bars->ds_smem_full);
         }
         if (ok && !mbar_wait_warp(&bars->acc_done, 0, abort_flag, budget_ns)) ok = false;
         if (ok) {
@@ -398,7 +426,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
-    } else if (!aborted_early && warp >= 8) {
+    } else if (!aborted_early && warp >= kWarpDq && warp < kWarpDq + 4) {
         // ------------------------------------------------ dQ warpgroup
         // Thread r owns query row r of the tile (its TMEM lane). Once the dQ
         // MMA has completed, the dS tile is free until the P/dS warpgroup
@@ -406,7 +434,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // 32-column segment at a time, in the 128-byte swizzled layout of the
         // accumulator's tensor map, and one lane hands each segment to the
         // TMA engine as a tiled reduce-add; rows past n are clipped by the TMA.
-        const int r = threadIdx.x - 256;
+        const int r = threadIdx.x - 32 * kWarpDq;
         const int wq = warp & 3;
         const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
         uint8_t* stage = smem + C::kOffdS + wq * C::kStageWarpBytes;
@@ -418,30 +446,37 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 break;
             }
             tc_fence_after();
-            uint32_t v[D];
+            // 64 columns at a time; the TMEM columns are released (dq_free)
+            // as soon as the last of them is in registers.
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c)
-                tmem_ld32(tl + C::kColdQ + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(v + 32 * c));
-            tmem_ld_wait();
-            tc_fence_before();
-            mbar_arrive(&bars->dq_free);
-#pragma unroll
-            for (int g = 0; g < D / 32; ++g) {
-                uint8_t* buf = stage + (g & 1) * 4096;
-                if (g >= 2) {
-                    if (lane == 0) bulk_wait_group_read1();   // buffer g-2 read
-                    __syncwarp();
+            for (int pair = 0; pair < D / 64; ++pair) {
+                uint32_t v[64];
+                tmem_ld32(tl + C::kColdQ + 64 * pair, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_ld32(tl + C::kColdQ + 64 * pair + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                tmem_ld_wait();
+                if (pair == D / 64 - 1) {
+                    tc_fence_before();
+                    mbar_arrive(&bars->dq_free);
                 }
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                        make_uint4(v[32 * g + 4 * k], v[32 * g + 4 * k + 1], v[32 * g + 4 * k + 2],
-                                   v[32 * g + 4 * k + 3]);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_reduce_add_3d(&tmdQacc, buf, 32 * g, row0, bh);
-                    bulk_commit_group();
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int g = 2 * pair + hh;                  // columns 32g..32g+31
+                    uint8_t* buf = stage + hh * 4096;
+                    if (g >= 2) {
+                        if (lane == 0) bulk_wait_group_read1();   // buffer's previous segment read
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                            make_uint4(v[32 * hh + 4 * k], v[32 * hh + 4 * k + 1],
+                                       v[32 * hh + 4 * k + 2], v[32 * hh + 4 * k + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_3d(&tmdQacc, buf, 32 * g, row0, bh);
+                        bulk_commit_group();
+                    }
                 }
             }
             if (lane == 0) bulk_wait_group_read0();
@@ -458,7 +493,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
