@@ -1,6 +1,7 @@
 // attn.cu -- the C ABI declared in include/attn.h: argument checks, workspace
 // carving, TMA descriptors, kernel-path choice and launches. All kernels are
 // compiled into this one translation unit.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -157,6 +158,20 @@ inline attn_status_t launched() {
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Number of SMs of the current device (cached per device).
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+            v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
 int grid_for(size_t work_items, int per_block, int cap) {
     size_t g = (work_items + per_block - 1) / per_block;
     if (g < 1) g = 1;
@@ -265,21 +280,26 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
                          void* dV, int BH, int n, int m, int causal, float scale,
                          cudaStream_t st) {
     using C = attn::bwdtc::Cfg<D>;
-    CUtensorMap mq, mk, mv, mdo, mdq;
+    CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
     if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) ||
         !make_map(&mv, V, D, m, BH) || !make_map(&mdo, dO, D, n, BH) ||
-        !make_map_typed(&mdq, dQacc, D, n, BH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 32, 32))
+        !make_map_typed(&mdq, dQacc, D, n, BH, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 32, 32) ||
+        !make_map_typed(&mdk, dK, D, m, BH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, 32) ||
+        !make_map_typed(&mdv, dV, D, m, BH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, 32))
         return ATTN_ERR_CUDA;
     auto kern = attn::bwdtc::bwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return ATTN_ERR_CUDA;
-    const long long grid = static_cast<long long>((m + kTile - 1) / kTile) * BH;
+    const int num_kt = (m + kTile - 1) / kTile;
+    const long long grid = static_cast<long long>(num_kt) * BH;
+    // heads per scheduling group: about 256 CTAs a group
+    const int head_group = std::max(1, std::min(BH, 256 / num_kt));
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mdo, mdq, lse2, Dd, n_pad, dQacc, static_cast<__nv_bfloat16*>(dK),
-            static_cast<__nv_bfloat16*>(dV), n, m, BH, causal, scale, scale * kLog2e,
-            kWaitBudgetNs);
+            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, n_pad, n, m, BH, head_group, sm_count(),
+            causal, scale,
+            scale * kLog2e, kWaitBudgetNs);
         return launched();
     });
 }

@@ -110,21 +110,21 @@ struct Bars {
     int abort;
 };
 
-// One 32-query chunk c of a P/dS warpgroup: P^T and dS^T from the S^T / dP^T
-// values in registers, written back to TMEM over the first 16 of the chunk's
-// own 32 S^T / dP^T columns; the packed dS is returned in `dk` for the shared
-// memory tile.
-template <int D>
-__device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const uint32_t (&pr)[32],
-                                          const float* lse_s, const float* dd_s, bool masked,
-                                          int keys_masked_below, float scale, float scale_log2,
-                                          uint32_t tmem_lane, uint32_t (&dk)[16]) {
-    using C = Cfg<D>;
-    uint32_t pk[16];
+// Sixteen queries (columns q0..q0+15 of a tile) for one key row: P^T and dS^T
+// from the S^T / dP^T values in registers. P^T and dS^T are written back to
+// TMEM at `pcol` / `dscol` (8 columns each, two bf16 per column); the packed
+// dS is also returned in `dk` for the shared-memory tile. MASKED applies the
+// causal / key-range mask: columns below `keys_masked_below` get P = 0.
+template <bool MASKED>
+__device__ __forceinline__ void pds_half(int q0, const uint32_t (&sr)[16], const uint32_t (&pr)[16],
+                                         const float* lse_s, const float* dd_s,
+                                         int keys_masked_below, float scale, float scale_log2,
+                                         uint32_t pcol, uint32_t dscol, uint32_t* dk) {
+    uint32_t pk[8];
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-        const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + 4 * g);
-        const float4 d4 = *reinterpret_cast<const float4*>(dd_s + c * 32 + 4 * g);
+    for (int g = 0; g < 4; ++g) {
+        const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q0 + 4 * g);
+        const float4 d4 = *reinterpret_cast<const float4*>(dd_s + q0 + 4 * g);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
         const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
         float p[4], ds[4];
@@ -132,7 +132,7 @@ __device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const
         for (int h = 0; h < 4; ++h) {
             const int e = 4 * g + h;
             p[h] = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, -lv[h]));
-            if (masked && (c * 32 + e) < keys_masked_below) p[h] = 0.f;
+            if (MASKED && (q0 + e) < keys_masked_below) p[h] = 0.f;
             ds[h] = p[h] * fmaf(__uint_as_float(pr[e]), scale, -dv[h]);
         }
         pk[2 * g] = pack_bf16x2(p[0], p[1]);
@@ -140,8 +140,8 @@ __device__ __forceinline__ void pds_chunk(int c, const uint32_t (&sr)[32], const
         dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
         dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
     }
-    tmem_st16(tmem_lane + C::kColP + c * 32, pk);
-    tmem_st16(tmem_lane + C::kColdS + c * 32, dk);
+    tmem_st8(pcol, pk);
+    tmem_st8(dscol, dk);
 }
 
 // dS of chunk c for key row r into the shared tile (queries contiguous,
@@ -158,23 +158,37 @@ __device__ __forceinline__ void store_ds_chunk(uint8_t* sdS, int c, int r, const
     }
 }
 
+// The (head, key tile) of CTA `b` in launch order (see the kernel's comment).
+__device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int& bh, int& kt) {
+    const int group = b / (hg * num_kt);
+    const int within = b % (hg * num_kt);
+    const int heads_here = min(hg, BH - group * hg);
+    kt = within / heads_here;
+    bh = group * hg + within % heads_here;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-           const __grid_constant__ CUtensorMap tmdQacc, const float* __restrict__ lse2, const float* __restrict__ Dd, int n_pad,
-           float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dK,
-           __nv_bfloat16* __restrict__ dV, int n, int m, int BH, int causal, float scale,
-           float scale_log2, unsigned long long budget_ns) {
+           const __grid_constant__ CUtensorMap tmdQacc, const __grid_constant__ CUtensorMap tmdK,
+           const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ lse2, const float* __restrict__ Dd, int n_pad,
+           int n, int m, int BH, int head_group,
+           int prefetch_stride, int causal, float scale, float scale_log2,
+           unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA order: heads in groups of `hg` (about 256 CTAs a group, so the
+    // heads in flight keep their Q/dO tiles and dQ rows in L2); inside a group
+    // key-tile major, so the longest CTAs of the group (lowest key tiles, if
+    // causal) start first and the shortest run last.
     const int num_kt = (m + kBN - 1) / kBN;
-    const int bh = int(blockIdx.x / num_kt);  // head-major: one head's key tiles together,
-    const int kt = int(blockIdx.x % num_kt);  // the longest (lowest, if causal) first
+    int bh, kt;
+    cta_tile(int(blockIdx.x), num_kt, BH, head_group, bh, kt);
     const int k0 = kt * kBN;
     const int num_qt = (n + kBM - 1) / kBM;
     const int first_qt = causal ? kt : 0;
@@ -218,10 +232,22 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         prefetch_tensor_map(&tmV);
         prefetch_tensor_map(&tmdO);
         prefetch_tensor_map(&tmdQacc);
+        prefetch_tensor_map(&tmdK);
+        prefetch_tensor_map(&tmdV);
         mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p) {
             tma_load_3d(smem + C::kOffK + p * C::kPanelBytes, &tmK, &bars->kv_full, p * 64, k0, bh);
             tma_load_3d(smem + C::kOffV + p * C::kPanelBytes, &tmV, &bars->kv_full, p * 64, k0, bh);
+        }
+        // Warm L2 with the K/V tiles of the CTA that will most likely start on
+        // a free SM about one CTA lifetime from now.
+        if (int(blockIdx.x) + prefetch_stride < int(gridDim.x)) {
+            int nbh, nkt;
+            cta_tile(int(blockIdx.x) + prefetch_stride, num_kt, BH, head_group, nbh, nkt);
+            for (int p = 0; p < C::kPanels; ++p) {
+                tma_prefetch_l2_3d(&tmK, p * 64, nkt * kBN, nbh);
+                tma_prefetch_l2_3d(&tmV, p * 64, nkt * kBN, nbh);
+            }
         }
         int issued = 0;
         for (int t = 0; t < T; ++t) {
@@ -357,31 +383,50 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const float* dd_s = reinterpret_cast<const float*>(smem + C::kOffDd + s * kBM * 4);
             // Keys past the end get P = 0 in every column; on the diagonal tile,
             // key r is masked for the queries in the tile before it (q < r).
+            // The masked variant is chosen per warp, never per lane: it holds
+            // warp-collective tcgen05.st instructions, which must not sit in a
+            // divergent branch. Lanes that need no mask get a bound of 0.
             const bool diag = causal && (q0 == k0);
-            const bool masked = !key_ok || diag;
-            const int below = key_ok ? r : kBM;
+            const int below = !key_ok ? kBM : (diag ? r : 0);
+            const bool masked = __any_sync(0xffffffffu, below > 0);
+            // Four half-chunks of 16 queries (two chunks), each half's TMEM
+            // loads issued while the previous half is computed. A chunk's
+            // P^T/dS^T go into the first 16 of its own 32 columns: half h of
+            // chunk c writes columns 32c+8h..32c+8h+7, which it has read.
             uint32_t ds0[16], ds1[16];
-            {
-                const int c = 2 * grp;
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tl + C::kColS + c * 32, sr);
-                tmem_ld32(tl + C::kColdP + c * 32, pr);
-                tmem_ld_wait();
-                pds_chunk<D>(c, sr, pr, lse_s, dd_s, masked, below, scale, scale_log2, tl, ds0);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars->ds_chunk[c]);
-            }
-            {
-                const int c = 2 * grp + 1;
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tl + C::kColS + c * 32, sr);
-                tmem_ld32(tl + C::kColdP + c * 32, pr);
-                tmem_ld_wait();
-                pds_chunk<D>(c, sr, pr, lse_s, dd_s, masked, below, scale, scale_log2, tl, ds1);
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars->ds_chunk[c]);
+            uint32_t sA[16], pA[16], sB[16], pB[16];
+            const int cbase = 2 * grp;
+            tmem_ld16(tl + C::kColS + cbase * 32, sA);
+            tmem_ld16(tl + C::kColdP + cbase * 32, pA);
+            tmem_ld_wait();
+#pragma unroll
+            for (int hc = 0; hc < 4; ++hc) {
+                const int c = cbase + (hc >> 1), half = hc & 1;
+                const int qcol = 32 * c + 16 * half;              // first query of the half
+                uint32_t (&scur)[16] = (hc & 1) ? sB : sA;
+                uint32_t (&pcur)[16] = (hc & 1) ? pB : pA;
+                uint32_t (&snxt)[16] = (hc & 1) ? sA : sB;
+                uint32_t (&pnxt)[16] = (hc & 1) ? pA : pB;
+                if (hc < 3) {
+                    const int qn = 32 * (cbase + ((hc + 1) >> 1)) + 16 * ((hc + 1) & 1);
+                    tmem_ld16(tl + C::kColS + qn, snxt);
+                    tmem_ld16(tl + C::kColdP + qn, pnxt);
+                }
+                uint32_t* dk = ((hc >> 1) ? ds1 : ds0) + 8 * half;
+                const uint32_t pcol = tl + C::kColP + 32 * c + 8 * half;
+                const uint32_t dscol = tl + C::kColdS + 32 * c + 8 * half;
+                if (masked)
+                    pds_half<true>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
+                                   dscol, dk);
+                else
+                    pds_half<false>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
+                                    dscol, dk);
+                if (half == 1) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bars->ds_chunk[c]);
+                }
+                if (hc < 3) tmem_ld_wait();
             }
             // The dS tile doubles as the dQ warpgroup's staging buffer for the
             // previous tile: write it once the TMA engine has read that.
@@ -395,33 +440,40 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             fence_proxy_async_smem();
             mbar_arrive(&bars->ds_smem_full);
         }
+        // Epilogue: group 0 writes dV, group 1 writes dK. Each warp converts
+        // its 32 rows to bf16 in the 128-byte swizzled layout of the output's
+        // tensor map, staged in this CTA's Q / dO stage buffers (every MMA
+        // that read them is complete once acc_done has fired), and one lane
+        // stores 32 x 64 boxes with the TMA; rows past m are clipped.
         if (ok && !mbar_wait_warp(&bars->acc_done, 0, abort_flag, budget_ns)) ok = false;
         if (ok) {
             tc_fence_after();
-            __nv_bfloat16* vrow = dV + (size_t(bh) * m + j) * D;
-            __nv_bfloat16* krow = dK + (size_t(bh) * m + j) * D;
+            const uint32_t col = grp == 0 ? C::kColdV : C::kColdK;
+            const CUtensorMap* out_map = grp == 0 ? &tmdV : &tmdK;
+            uint8_t* stage = smem + (grp == 0 ? C::kOffQ : C::kOffdO) + (warp & 3) * (32 * D * 2);
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? C::kColdV : C::kColdK;
-                __nv_bfloat16* dst = which == 0 ? vrow : krow;
+            for (int pnl = 0; pnl < C::kPanels; ++pnl) {
+                uint32_t rr[64];
+                tmem_ld32(tl + col + 64 * pnl, *reinterpret_cast<uint32_t(*)[32]>(rr));
+                tmem_ld32(tl + col + 64 * pnl + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
+                tmem_ld_wait();
+                uint8_t* buf = stage + pnl * 4096;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t rr[32];
-                    tmem_ld32(tl + col + c * 32, rr);
-                    tmem_ld_wait();
-                    if (key_ok) {
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]), __uint_as_float(rr[8 * v + 1]));
-                            w.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]), __uint_as_float(rr[8 * v + 3]));
-                            w.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]), __uint_as_float(rr[8 * v + 5]));
-                            w.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]), __uint_as_float(rr[8 * v + 7]));
-                            *reinterpret_cast<uint4*>(dst + c * 32 + 8 * v) = w;
-                        }
-                    }
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) = make_uint4(
+                        pack_bf16x2(__uint_as_float(rr[8 * k + 0]), __uint_as_float(rr[8 * k + 1])),
+                        pack_bf16x2(__uint_as_float(rr[8 * k + 2]), __uint_as_float(rr[8 * k + 3])),
+                        pack_bf16x2(__uint_as_float(rr[8 * k + 4]), __uint_as_float(rr[8 * k + 5])),
+                        pack_bf16x2(__uint_as_float(rr[8 * k + 6]), __uint_as_float(rr[8 * k + 7])));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(out_map, buf, 64 * pnl, k0 + 32 * (warp & 3), bh);
+                    bulk_commit_group();
                 }
             }
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
         } else {
             record_device_error(kErrTimeout);
             *abort_flag = 1;
@@ -483,7 +535,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             __syncwarp();
             mbar_arrive(&bars->ds_smem_free);
         }
-        if (lane == 0) bulk_wait_group0();
+        // The CTA may exit once the TMA has read its shared-memory sources;
+        // the reduce-adds themselves complete before the grid does.
+        if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
         if (!ok) {
             record_device_error(kErrTimeout);

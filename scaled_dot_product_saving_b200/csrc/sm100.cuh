@@ -11,6 +11,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "exp2_poly.h"
+
 namespace attn {
 
 // Device error word (one per device); written by kernels that give up a wait.
@@ -141,6 +143,18 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const 
         "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+// Tiled 3-D store shared -> global through a tensor map, tracked by this
+// thread's bulk async-group. Elements of the box outside the tensor are not
+// written; coordinates are never negative here.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1,
+                                             int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_addr(src)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // Wait until at most one of this thread's committed bulk groups is still
 // reading its shared-memory source.
 __device__ __forceinline__ void bulk_wait_group_read1() {
@@ -168,6 +182,14 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 // Wait until this thread's committed bulk groups have fully completed.
 __device__ __forceinline__ void bulk_wait_group0() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Prefetch a tile of a tensor into L2 (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* map) {
@@ -275,6 +297,25 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+// TMEM -> registers: 32 lanes x 32 bit, 16 consecutive columns per thread.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Registers -> TMEM: 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
 // Registers -> TMEM: 16 consecutive columns per thread.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
@@ -313,6 +354,23 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Base-2 exponential on the FMA pipe, to share the work of the MUFU unit:
+// Cody-Waite reduction 2^x = 2^n * 2^f with n = round(x) (the 1.5 * 2^23
+// rounding trick) and f in [-1/2, 1/2], 2^f from the minimax polynomial of
+// exp2_poly.h, and n added to the result's exponent field. Relative error at
+// most exp2poly::kMaxRelError (7.5e-5) for x in (-126, 0.5]; inputs at or
+// below -126 are clamped there and give a value no larger than 2^-125 rather
+// than 0 -- callers that need an exact zero (masked scores) set it themselves.
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -126.0f);
+    const float t = x + 12582912.0f;
+    const float f = x - (t - 12582912.0f);
+    float p = fmaf(exp2poly::kC3, f, exp2poly::kC2);
+    p = fmaf(p, f, exp2poly::kC1);
+    p = fmaf(p, f, exp2poly::kC0);
+    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
