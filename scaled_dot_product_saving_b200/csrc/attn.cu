@@ -200,18 +200,20 @@ template <int D>
 attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, float* LSE,
                          int BH, int n, int m, int causal, float scale, cudaStream_t st) {
     using C = attn::fwdtc::Cfg<D>;
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) || !make_map(&mv, V, D, m, BH))
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) || !make_map(&mv, V, D, m, BH) ||
+        !make_map_typed(&mo, O, D, n, BH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, 32))
         return ATTN_ERR_CUDA;
     auto kern = attn::fwdtc::fwd_kernel<D>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return ATTN_ERR_CUDA;
-    const long long grid = static_cast<long long>((n + kTile - 1) / kTile) * BH;
+    // One CTA per pair of query tiles (p, num_qt - 1 - p) of one head.
+    const int num_qt = (n + attn::fwdtc::kBM - 1) / attn::fwdtc::kBM;
+    const long long grid = static_cast<long long>((num_qt + 1) / 2) * BH;
     return traced(ATTN_KERNEL_FWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, static_cast<__nv_bfloat16*>(O), LSE, n, m, BH, causal, scale * kLog2e,
-            kWaitBudgetNs);
+            mq, mk, mv, mo, LSE, n, m, causal, scale * kLog2e, kWaitBudgetNs);
         return launched();
     });
 }

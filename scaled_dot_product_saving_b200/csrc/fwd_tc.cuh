@@ -1,23 +1,43 @@
 // fwd_tc.cuh -- tensor-core forward for bf16, d == dv in {64, 128}.
 //
-// One CTA computes a 128-row query tile of one (batch, head) and walks the
-// key/value tiles (128 keys each; only tiles at or below the diagonal when
-// causal):
-//   S = Q K_t^T                     tcgen05.mma, A = Q, B = K_t (both K-major
-//                                   in shared memory), fp32 D in TMEM
-//   running max / sum, P = 2^(S*scale*log2e - max)   128 softmax threads,
-//                                   one query row (TMEM lane) each
-//   O += P V_t                      tcgen05.mma, A = P read from TMEM (bf16
-//                                   written over its own S columns),
-//                                   B = V_t (MN-major), O in TMEM
-// At the end O / sum goes to global memory as bf16 and the row's log-sum-exp
-// (natural log) as fp32. The running max is only raised, and O rescaled, when
-// a new row max exceeds the one in use by more than 2^8 in P.
+// Computes O = softmax(scale * Q K^T) V and the row log-sum-exp (the forward
+// whose softmax statistics the backward recomputes P from: "Attention Backward
+// Pass (dQ, dK, dV)", section on the forward; under the causal mask key j > i
+// is excluded before the softmax).
 //
-// Warp roles (256 threads): warp 0 = TMA producer, warp 1 = TMEM allocator
-// and MMA issuer, warps 4-7 = softmax (warp 4+w owns TMEM lanes 32w..32w+31).
-// S is double-buffered in TMEM so that the tensor cores compute S_{t+1}
-// while the softmax threads work on S_t.
+// One CTA computes two 128-row query tiles, A and B, of one (batch, head),
+// sharing every key and value tile it loads. Query tiles are paired zig-zag
+// (tile p with tile num_qt - 1 - p), so under the causal mask every CTA walks
+// the same number of key tiles. For each 128-key tile t and each query tile x:
+//   S_x = Q_x K_t^T          tcgen05.mma, both operands K-major in shared
+//                            memory, fp32 accumulator in TMEM
+//   P_x = 2^(S_x * scale * log2e - m_x)   one softmax warpgroup per query
+//                            tile, one row (TMEM lane) per thread, m_x the
+//                            running row maximum in use
+//   O_x += P_x V_t           tcgen05.mma, A = P_x read from TMEM (bf16,
+//                            written over the S_x columns it came from),
+//                            B = V_t (MN-major), O_x in TMEM
+// The MMA thread issues PV_A(t), S_A(t+1), PV_B(t), S_B(t+1), ... so that the
+// tensor cores work on one tile while the other tile's softmax runs. Because
+// S_x(t+1) is issued after PV_x(t) by the same thread, the barrier that reports
+// S_x(t+1) also reports PV_x(t) complete: the softmax may rescale O_x as soon as
+// it sees S_x(t+1).
+//
+// The running maximum is raised, and O rescaled, only when a tile's row
+// maximum exceeds the one in use by more than 2^8 in P, so P <= 256 and the
+// row sum stays well inside fp32. A share of the exponentials is computed on
+// the FMA pipe (exp2_fma_x2) to relieve the MUFU unit; the scaled scores and
+// the row sums use the paired fp32 instructions. At the end O / sum is stored
+// as bf16 through shared memory with the TMA, and the row's natural-log LSE as
+// fp32.
+//
+// Warp roles (320 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of
+// tile B (warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31), warp 8 TMA producer,
+// warp 9 TMEM allocator and MMA issuer.
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
+// O_B [256+d, 256+2d).
+// Shared memory: Q_A, Q_B, then K and V rings with their own barriers (a K
+// tile is released as soon as both S products that read it are done).
 #pragma once
 
 #include "sm100.cuh"
@@ -25,47 +45,96 @@
 namespace attn {
 namespace fwdtc {
 
-constexpr int kBM = 128;      // queries per CTA
+constexpr int kBM = 128;      // queries per tile
 constexpr int kBN = 128;      // keys per tile
-constexpr int kThreads = 256;
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kThreads = 320;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Pairs of a 32-key chunk (bit e = pair e) whose exponentials use the FMA pipe.
+constexpr uint32_t kPolyPairs = 0x8888u;
 
 template <int D>
 struct Cfg {
-    static constexpr int kStages = (D == 64) ? 4 : 2;
+    static constexpr int kKStages = (D == 64) ? 4 : 3;
+    static constexpr int kVStages = (D == 64) ? 4 : 2;
     static constexpr int kPanels = D / 64;              // 64-column swizzle panels
     static constexpr int kTileBytes = kBM * D * 2;      // a 128-row bf16 tile
     static constexpr int kPanelBytes = kBM * 128;       // 128 rows x 128 B
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
-    static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr int kBarBytes = 256;
-    static constexpr int kSmemBytes = kOffBar + kBarBytes;
-    // TMEM columns (512 allocated): two S buffers of 128 fp32 columns, then O.
+    static constexpr int kOffQ = 0;                     // Q_A, Q_B
+    static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+    static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+    static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+    static constexpr int kSmemBytes = kOffBar + 256;
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+    static constexpr uint32_t kColS0 = 0;                // S_x at kColS0 + 128 x
+    static constexpr uint32_t kColO0 = 256;              // O_x at kColO0 + D x
+    static constexpr int kStageWarpBytes = 32 * D * 2;  // epilogue: 32 rows per warp
 };
+static_assert(Cfg<128>::kSmemBytes <= 232448, "shared memory");
 
 struct Bars {
     uint64_t q_full;
-    uint64_t kv_full[4];
-    uint64_t kv_empty[4];
+    uint64_t k_full[4];
+    uint64_t k_empty[4];
+    uint64_t v_full[4];
+    uint64_t v_empty[4];
     uint64_t s_full[2];
     uint64_t p_full[2];
-    uint64_t o_done;
+    uint64_t o_done[2];
     uint64_t mma_drain;
     uint32_t tmem_base;
     int abort;
 };
 
+// Maximum (or, for a negative scale, minimum) of a 32-key chunk of raw scores,
+// excluding keys after `kmax` when MASKED.
+template <bool NEG, bool MASKED>
+__device__ __forceinline__ float chunk_extreme(const uint32_t (&r)[32], float acc, int key0,
+                                               int kmax) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float a = __uint_as_float(r[e]), b = __uint_as_float(r[e + 1]);
+        if (MASKED) {
+            if (key0 + e > kmax) a = NEG ? INFINITY : -INFINITY;
+            if (key0 + e + 1 > kmax) b = NEG ? INFINITY : -INFINITY;
+        }
+        acc = NEG ? fmin3(acc, a, b) : fmax3(acc, a, b);
+    }
+    return acc;
+}
+
+// P for a 32-key chunk: 2^(raw * scale_log2 - m) (exactly 0 for masked keys),
+// packed to bf16 pairs in `pk`, summed into `sum`.
+template <bool MASKED>
+__device__ __forceinline__ void chunk_p(const uint32_t (&r)[32], f32x2 sl2, f32x2 neg_m,
+                                        int key0, int kmax, f32x2& sum, uint32_t (&pk)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float2 x = split_f32x2(
+            fma_x2(make_f32x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sl2, neg_m));
+        float2 p;
+        if ((kPolyPairs >> e) & 1u) {
+            p = exp2_fma_x2(x.x, x.y);
+        } else {
+            p.x = ex2(x.x);
+            p.y = ex2(x.y);
+        }
+        if (MASKED) {
+            if (key0 + 2 * e > kmax) p.x = 0.f;
+            if (key0 + 2 * e + 1 > kmax) p.y = 0.f;
+        }
+        sum = add_x2(sum, make_f32x2(p.x, p.y));
+        pk[e] = pack_bf16x2(p.x, p.y);
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-           const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
-           float* __restrict__ LSE, int n, int m, int BH, int causal, float scale_log2,
+           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+           float* __restrict__ LSE, int n, int m, int causal, float scale_log2,
            unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -74,11 +143,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_qt = (n + kBM - 1) / kBM;
-    const int qt = num_qt - 1 - int(blockIdx.x / BH);   // heaviest (last) query tiles first
-    const int bh = int(blockIdx.x % BH);
-    const int q0 = qt * kBM;
-    const int kv_end = causal ? min(m, q0 + kBM) : m;
-    const int num_kv = (kv_end + kBN - 1) / kBN;
+    const int num_pairs = (num_qt + 1) / 2;
+    const int bh = int(blockIdx.x) / num_pairs;   // CTAs of one head run together: K/V stay in L2
+    const int pair = int(blockIdx.x) % num_pairs;
+    const int num_kt = (m + kBN - 1) / kBN;
+    const bool has_b = num_qt - 1 - pair != pair;
+    // query tile and number of key tiles of tile A (x = 0) and tile B (x = 1)
+    const int qt_a = pair, qt_b = num_qt - 1 - pair;
+    const int nkv_a = causal ? min(num_kt, qt_a + 1) : num_kt;
+    const int nkv_b = has_b ? (causal ? min(num_kt, qt_b + 1) : num_kt) : 0;
+    auto qt_of = [&](int x) { return x ? qt_b : qt_a; };
+    auto nkv_of = [&](int x) { return x ? nkv_b : nkv_a; };
+    const int num_kv = max(nkv_a, nkv_b);
 
     if (threadIdx.x == 0) {
         // The swizzled tiles need a 1024-byte aligned base. A CTA that starts
@@ -87,19 +163,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (misaligned) record_device_error(kErrTimeout);
         bars->abort = (misaligned || *reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0) ? 1 : 0;
         mbar_init(&bars->q_full, 1);
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&bars->kv_full[s], 1);
-            mbar_init(&bars->kv_empty[s], 1);
+        for (int s = 0; s < 4; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->s_full[b], 1);
-            mbar_init(&bars->p_full[b], 128);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_full[x], 128);
+            mbar_init(&bars->o_done[x], 1);
         }
-        mbar_init(&bars->o_done, 1);
         mbar_init(&bars->mma_drain, 1);
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(&bars->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
@@ -109,76 +187,116 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const uint32_t tmem = bars->tmem_base;
     const bool aborted_early = bars->abort != 0;
 
-    if (!aborted_early && warp == 0 && lane == 0) {
+    if (!aborted_early && warp == kWarpProducer && lane == 0) {
         // ------------------------------------------------ TMA producer
         prefetch_tensor_map(&tmQ);
         prefetch_tensor_map(&tmK);
         prefetch_tensor_map(&tmV);
-        mbar_arrive_expect_tx(&bars->q_full, C::kTileBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(smem + C::kOffQ + p * C::kPanelBytes, &tmQ, &bars->q_full, p * 64, q0, bh);
-        int issued = 0;
+        prefetch_tensor_map(&tmO);
+        const int nq = has_b ? 2 : 1;
+        mbar_arrive_expect_tx(&bars->q_full, nq * C::kTileBytes);
+        for (int x = 0; x < nq; ++x)
+            for (int p = 0; p < C::kPanels; ++p)
+                tma_load_3d(smem + C::kOffQ + x * C::kTileBytes + p * C::kPanelBytes, &tmQ,
+                            &bars->q_full, p * 64, qt_of(x) * kBM, bh);
+        int k_issued = 0, v_issued = 0;
         for (int t = 0; t < num_kv; ++t) {
-            const int s = t % C::kStages, k = t / C::kStages;
-            if (t >= C::kStages &&
-                !mbar_wait(&bars->kv_empty[s], (k - 1) & 1, abort_flag, budget_ns)) {
-                record_device_error(kErrTimeout);
-                *abort_flag = 1;
+            const int sk = t % C::kKStages, sv = t % C::kVStages;
+            if (t >= C::kKStages &&
+                !mbar_wait(&bars->k_empty[sk], (t / C::kKStages - 1) & 1, abort_flag, budget_ns))
                 break;
-            }
-            mbar_arrive_expect_tx(&bars->kv_full[s], 2 * C::kTileBytes);
-            for (int p = 0; p < C::kPanels; ++p) {
-                tma_load_3d(smem + C::kOffK + s * C::kTileBytes + p * C::kPanelBytes, &tmK,
-                            &bars->kv_full[s], p * 64, t * kBN, bh);
-                tma_load_3d(smem + C::kOffV + s * C::kTileBytes + p * C::kPanelBytes, &tmV,
-                            &bars->kv_full[s], p * 64, t * kBN, bh);
-            }
-            ++issued;
+            mbar_arrive_expect_tx(&bars->k_full[sk], C::kTileBytes);
+            for (int p = 0; p < C::kPanels; ++p)
+                tma_load_3d(smem + C::kOffK + sk * C::kTileBytes + p * C::kPanelBytes, &tmK,
+                            &bars->k_full[sk], p * 64, t * kBN, bh);
+            ++k_issued;
+            if (t >= C::kVStages &&
+                !mbar_wait(&bars->v_empty[sv], (t / C::kVStages - 1) & 1, abort_flag, budget_ns))
+                break;
+            mbar_arrive_expect_tx(&bars->v_full[sv], C::kTileBytes);
+            for (int p = 0; p < C::kPanels; ++p)
+                tma_load_3d(smem + C::kOffV + sv * C::kTileBytes + p * C::kPanelBytes, &tmV,
+                            &bars->v_full[sv], p * 64, t * kBN, bh);
+            ++v_issued;
+        }
+        if (v_issued < num_kv) {
+            record_device_error(kErrTimeout);
+            *abort_flag = 1;
         }
         // Drain: every load issued must land before the CTA may exit. Tiles
-        // older than the last kStages were consumed, so they have landed.
+        // older than the last ring's worth were consumed, so they have landed.
         (void)mbar_wait_timed(&bars->q_full, 0, budget_ns);
-        for (int t = (issued > C::kStages ? issued - C::kStages : 0); t < issued; ++t)
-            (void)mbar_wait_timed(&bars->kv_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == 1 && lane == 0) {
+        for (int t = (k_issued > C::kKStages ? k_issued - C::kKStages : 0); t < k_issued; ++t)
+            (void)mbar_wait_timed(&bars->k_full[t % C::kKStages], (t / C::kKStages) & 1, budget_ns);
+        for (int t = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); t < v_issued; ++t)
+            (void)mbar_wait_timed(&bars->v_full[t % C::kVStages], (t / C::kVStages) & 1, budget_ns);
+    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
         // ------------------------------------------------ MMA issuer
         constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, 0, 0);
         constexpr uint32_t idO = idesc_bf16_f32(kBM, D, 0, 1);
-        const uint32_t sQ = smem_addr(smem + C::kOffQ);
-        bool ok = mbar_wait(&bars->q_full, 0, abort_flag, budget_ns);
-        auto issue_S = [&](int t) -> bool {
-            const int s = t % C::kStages;
-            if (!mbar_wait(&bars->kv_full[s], (t / C::kStages) & 1, abort_flag, budget_ns))
-                return false;
-            tc_fence_after();
-            const uint32_t sK = smem_addr(smem + C::kOffK + s * C::kTileBytes);
-            const uint32_t dS = tmem + ((t & 1) ? C::kColS1 : C::kColS0);
+        auto issue_S = [&](int x, int t) {
+            const uint32_t sQ = smem_addr(smem + C::kOffQ + x * C::kTileBytes);
+            const uint32_t sK = smem_addr(smem + C::kOffK + (t % C::kKStages) * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(dS, sdesc_sw128(sQ + koff, 16, 1024), sdesc_sw128(sK + koff, 16, 1024), idS,
-                       kk > 0);
+                mma_ss(tmem + C::kColS0 + 128 * x, sdesc_sw128(sQ + koff, 16, 1024),
+                       sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0);
             }
-            mma_commit(&bars->s_full[t & 1]);
-            return true;
+            mma_commit(&bars->s_full[x]);
         };
-        if (ok) ok = issue_S(0);
-        for (int t = 0; ok && t < num_kv; ++t) {
-            if (t + 1 < num_kv && !issue_S(t + 1)) { ok = false; break; }
-            if (!mbar_wait(&bars->p_full[t & 1], (t >> 1) & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const int s = t % C::kStages;
-            const uint32_t sV = smem_addr(smem + C::kOffV + s * C::kTileBytes);
-            const uint32_t aP = tmem + ((t & 1) ? C::kColS1 : C::kColS0);
+        auto issue_PV = [&](int x, int t) {
+            const uint32_t sV = smem_addr(smem + C::kOffV + (t % C::kVStages) * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_ts(tmem + C::kColO, aP + kk * 8,
+                mma_ts(tmem + C::kColO0 + D * x, tmem + C::kColS0 + 128 * x + kk * 8,
                        sdesc_sw128(sV + kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0));
-            mma_commit(&bars->kv_empty[s]);
-            mma_commit(&bars->o_done);
+        };
+        bool ok = mbar_wait(&bars->q_full, 0, abort_flag, budget_ns) &&
+                  mbar_wait(&bars->k_full[0], 0, abort_flag, budget_ns);
+        if (ok) {
+            tc_fence_after();
+            for (int x = 0; x < 2; ++x)
+                if (nkv_of(x) > 0) issue_S(x, 0);
+            mma_commit(&bars->k_empty[0]);
+        }
+        for (int t = 0; ok && t < num_kv; ++t) {
+            bool v_ready = false, k_ready = false;
+            for (int x = 0; x < 2; ++x) {
+                if (t >= nkv_of(x)) continue;
+                if (!mbar_wait(&bars->p_full[x], t & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (!v_ready) {
+                    if (!mbar_wait(&bars->v_full[t % C::kVStages], (t / C::kVStages) & 1,
+                                   abort_flag, budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    v_ready = true;
+                }
+                tc_fence_after();
+                issue_PV(x, t);
+                if (t + 1 < nkv_of(x)) {
+                    if (!k_ready) {
+                        const int t1 = t + 1;
+                        if (!mbar_wait(&bars->k_full[t1 % C::kKStages], (t1 / C::kKStages) & 1,
+                                       abort_flag, budget_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        k_ready = true;
+                        tc_fence_after();
+                    }
+                    issue_S(x, t + 1);
+                } else {
+                    mma_commit(&bars->o_done[x]);   // last product into O_x
+                }
+            }
+            if (!ok) break;
+            if (k_ready) mma_commit(&bars->k_empty[(t + 1) % C::kKStages]);
+            mma_commit(&bars->v_empty[t % C::kVStages]);
         }
         if (!ok) {
             record_device_error(kErrTimeout);
@@ -187,42 +305,52 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // Drain: all MMAs issued here complete before TMEM is released.
         mma_commit(&bars->mma_drain);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
-    } else if (!aborted_early && warp >= 4) {
-        // ------------------------------------------------ softmax warpgroup
-        const int r = threadIdx.x - 128;               // query row in the tile == TMEM lane
-        const uint32_t lane_sel = uint32_t((warp & 3) * 32) << 16;
+    } else if (!aborted_early && warp < 8) {
+        // ------------------------------------------------ softmax warpgroups
+        const int x = warp >> 2;                         // query tile A or B
+        const int r = threadIdx.x & 127;                 // row in the tile == TMEM lane
+        const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16);
+        const uint32_t tS = tl + C::kColS0 + 128 * x, tO = tl + C::kColO0 + D * x;
+        const int q0 = qt_of(x) * kBM;
         const int row = q0 + r;
+        const int ntile = nkv_of(x);
+        const bool neg = scale_log2 < 0.f;
+        const f32x2 sl2 = make_f32x2(scale_log2, scale_log2);
+        // Keys after kmax are masked: past the end, or after the row (causal).
+        const int kmax = causal ? min(row, m - 1) : m - 1;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        for (int t = 0; t < num_kv; ++t) {
-            if (!mbar_wait_warp(&bars->s_full[t & 1], (t >> 1) & 1, abort_flag, budget_ns)) {
+        for (int t = 0; t < ntile; ++t) {
+            if (!mbar_wait_warp(&bars->s_full[x], t & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t tS = tmem + lane_sel + ((t & 1) ? C::kColS1 : C::kColS0);
-            float sv[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(tS + c * 32, rr);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(rr[e]) * scale_log2;
-            }
             const int k0 = t * kBN;
-            const bool need_mask = (k0 + kBN > m) || (causal && k0 + kBN - 1 > q0);
-            if (need_mask) {
+            const bool masked = __any_sync(0xffffffffu, k0 + kBN - 1 > kmax);
+            // pass 1: extreme raw score of the row over this key tile
+            float ext = neg ? INFINITY : -INFINITY;
 #pragma unroll
-                for (int e = 0; e < kBN; ++e) {
-                    const int key = k0 + e;
-                    if (key >= m || (causal && key > row)) sv[e] = -INFINITY;
+            for (int h = 0; h < 2; ++h) {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(tS + 64 * h, ra);
+                tmem_ld32(tS + 64 * h + 32, rb);
+                tmem_ld_wait(ra);
+                tmem_ld_wait(rb);
+                const int key0 = k0 + 64 * h;
+                if (neg) {
+                    ext = masked ? chunk_extreme<true, true>(ra, ext, key0, kmax)
+                                 : chunk_extreme<true, false>(ra, ext, key0, kmax);
+                    ext = masked ? chunk_extreme<true, true>(rb, ext, key0 + 32, kmax)
+                                 : chunk_extreme<true, false>(rb, ext, key0 + 32, kmax);
+                } else {
+                    ext = masked ? chunk_extreme<false, true>(ra, ext, key0, kmax)
+                                 : chunk_extreme<false, false>(ra, ext, key0, kmax);
+                    ext = masked ? chunk_extreme<false, true>(rb, ext, key0 + 32, kmax)
+                                 : chunk_extreme<false, false>(rb, ext, key0 + 32, kmax);
                 }
             }
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int e = 0; e < kBN; ++e) tmax = fmaxf(tmax, sv[e]);
-            const float m_new = fmaxf(m_run, tmax);
+            const float m_new = fmaxf(m_run, ext * scale_log2);
             const bool want = m_new > m_run + kRescaleThreshold;   // true on the first tile
             const bool warp_rescale = __any_sync(0xffffffffu, want && t > 0);
             float alpha = 1.f;
@@ -232,68 +360,82 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 l_run *= alpha;
             }
             if (warp_rescale) {
-                // O must hold P_{t-1} V_{t-1} before it is rescaled.
-                if (!mbar_wait_warp(&bars->o_done, (t - 1) & 1, abort_flag, budget_ns)) ok = false;
-                tc_fence_after();
-                const uint32_t tO = tmem + lane_sel + C::kColO;
+                // O_x holds P(t-1) V(t-1): S_x(t) was issued after that product.
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t rr[32];
                     tmem_ld32(tO + c * 32, rr);
-                    tmem_ld_wait();
+                    tmem_ld_wait(rr);
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
                     tmem_st32(tO + c * 32, rr);
                 }
             }
-            const float msub = (m_run == -INFINITY) ? 0.f : m_run;
-            float lsum = 0.f;
+            // pass 2: P as bf16 over the S columns already read (chunk c's P
+            // goes to columns 16c .. 16c+15, all read by then)
+            const f32x2 neg_m = make_f32x2(-m_run, -m_run);
+            f32x2 sum = make_f32x2(0.f, 0.f);
+            uint32_t ra[32], rb[32];
+            tmem_ld32(tS, ra);
 #pragma unroll
             for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+                uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+                tmem_ld_wait(cur);
+                if (c + 1 < kBN / 32) tmem_ld32(tS + 32 * (c + 1), nxt);
                 uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float p0 = ex2(sv[c * 32 + 2 * e] - msub);
-                    const float p1 = ex2(sv[c * 32 + 2 * e + 1] - msub);
-                    lsum += p0 + p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(tS + c * 16, pk);     // P over S columns already read
+                if (masked)
+                    chunk_p<true>(cur, sl2, neg_m, k0 + 32 * c, kmax, sum, pk);
+                else
+                    chunk_p<false>(cur, sl2, neg_m, k0 + 32 * c, kmax, sum, pk);
+                tmem_st16(tS + 16 * c, pk);
             }
-            l_run += lsum;
+            const float2 s2 = split_f32x2(sum);
+            l_run += s2.x + s2.y;
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[t & 1]);
-            if (!ok) break;
+            mbar_arrive(&bars->p_full[x]);
         }
-        if (ok && num_kv > 0 &&
-            !mbar_wait_warp(&bars->o_done, (num_kv - 1) & 1, abort_flag, budget_ns))
+        if (ok && ntile > 0 && !mbar_wait_warp(&bars->o_done[x], 0, abort_flag, budget_ns))
             ok = false;
-        if (ok) {
+        if (ok && ntile > 0) {
+            // Epilogue: O / sum as bf16, staged per warp (32 rows) in the
+            // 128B-swizzled layout of O's tensor map inside this tile's Q buffer
+            // (no MMA reads it any more), stored with the TMA; rows past n are
+            // clipped by the tensor map. LSE in natural log.
             tc_fence_after();
             const float inv = 1.f / l_run;
-            const uint32_t tO = tmem + lane_sel + C::kColO;
-            __nv_bfloat16* orow = O + (size_t(bh) * n + row) * D;
+            uint8_t* stage = smem + C::kOffQ + x * C::kTileBytes + (warp & 3) * C::kStageWarpBytes;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t rr[32];
-                tmem_ld32(tO + c * 32, rr);
-                tmem_ld_wait();
-                if (row < n) {
+            for (int pnl = 0; pnl < C::kPanels; ++pnl) {
+                uint32_t ra[32], rb[32];
+                tmem_ld32(tO + 64 * pnl, ra);
+                tmem_ld32(tO + 64 * pnl + 32, rb);
+                tmem_ld_wait(ra);
+                tmem_ld_wait(rb);
+                uint8_t* buf = stage + pnl * 4096;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(rr[8 * v + 0]) * inv, __uint_as_float(rr[8 * v + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(rr[8 * v + 2]) * inv, __uint_as_float(rr[8 * v + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(rr[8 * v + 4]) * inv, __uint_as_float(rr[8 * v + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(rr[8 * v + 6]) * inv, __uint_as_float(rr[8 * v + 7]) * inv);
-                        *reinterpret_cast<uint4*>(orow + c * 32 + 8 * v) = w;
-                    }
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t* src = (k < 4) ? ra + 8 * k : rb + 8 * (k - 4);
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(src[0]) * inv, __uint_as_float(src[1]) * inv);
+                    w.y = pack_bf16x2(__uint_as_float(src[2]) * inv, __uint_as_float(src[3]) * inv);
+                    w.z = pack_bf16x2(__uint_as_float(src[4]) * inv, __uint_as_float(src[5]) * inv);
+                    w.w = pack_bf16x2(__uint_as_float(src[6]) * inv, __uint_as_float(src[7]) * inv);
+                    *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) = w;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&tmO, buf, 64 * pnl, q0 + 32 * (warp & 3), bh);
+                    bulk_commit_group();
                 }
             }
             if (row < n) LSE[size_t(bh) * n + row] = (m_run + log2f(l_run)) * kLn2;
-        } else {
+            if (lane == 0) bulk_wait_group_read0();
+            __syncwarp();
+        } else if (!ok) {
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
@@ -301,7 +443,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

@@ -344,6 +344,20 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// Same wait, tied to the 32 registers of one earlier tmem_ld32 so that no use
+// of them can be scheduled before it (their contents are undefined until
+// then).
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -356,21 +370,67 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Base-2 exponential on the FMA pipe, to share the work of the MUFU unit:
-// Cody-Waite reduction 2^x = 2^n * 2^f with n = round(x) (the 1.5 * 2^23
-// rounding trick) and f in [-1/2, 1/2], 2^f from the minimax polynomial of
-// exp2_poly.h, and n added to the result's exponent field. Relative error at
-// most exp2poly::kMaxRelError (7.5e-5) for x in (-126, 0.5]; inputs at or
-// below -126 are clamped there and give a value no larger than 2^-125 rather
-// than 0 -- callers that need an exact zero (masked scores) set it themselves.
-__device__ __forceinline__ float exp2_fma(float x) {
-    x = fmaxf(x, -126.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p = fmaf(exp2poly::kC3, f, exp2poly::kC2);
-    p = fmaf(p, f, exp2poly::kC1);
-    p = fmaf(p, f, exp2poly::kC0);
-    return __int_as_float(__float_as_int(p) + ((__float_as_int(t) - 0x4B400000) << 23));
+// Three-input maximum and minimum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Pairs of fp32 values in one 64-bit register for the paired FMA-pipe
+// instructions of sm_100 (each half rounded exactly as the scalar operation).
+struct f32x2 {
+    uint64_t v;
+};
+__device__ __forceinline__ f32x2 make_f32x2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 split_f32x2(f32x2 a) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(a.v));
+    return r;
+}
+__device__ __forceinline__ f32x2 fma_x2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return r;
+}
+__device__ __forceinline__ f32x2 add_x2(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
+
+// Base-2 exponential of a pair on the FMA pipe, to share the work of the MUFU
+// unit: Cody-Waite reduction 2^x = 2^n * 2^f with n = round(x) (adding and
+// subtracting 1.5 * 2^23 rounds to an integer) and f in [-1/2, 1/2], 2^f from
+// the minimax polynomial of exp2_poly.h (Horner, paired fused multiply-adds),
+// and n added to the result's exponent field. Relative error at most
+// exp2poly::kMaxRelError (7.5e-5) for x in (-126, 16]; inputs at or below -126
+// are clamped there and give a value no larger than 2^-125 rather than 0 --
+// callers that need an exact zero (masked scores) set it themselves.
+__device__ __forceinline__ float2 exp2_fma_x2(float x0, float x1) {
+    const f32x2 x = make_f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+    const f32x2 magic = make_f32x2(12582912.0f, 12582912.0f);
+    const f32x2 neg_magic = make_f32x2(-12582912.0f, -12582912.0f);
+    const f32x2 minus1 = make_f32x2(-1.0f, -1.0f);
+    const f32x2 t = add_x2(x, magic);
+    const f32x2 f = fma_x2(add_x2(t, neg_magic), minus1, x);
+    f32x2 p = fma_x2(make_f32x2(exp2poly::kC3, exp2poly::kC3), f,
+                     make_f32x2(exp2poly::kC2, exp2poly::kC2));
+    p = fma_x2(p, f, make_f32x2(exp2poly::kC1, exp2poly::kC1));
+    p = fma_x2(p, f, make_f32x2(exp2poly::kC0, exp2poly::kC0));
+    const float2 pp = split_f32x2(p), tt = split_f32x2(t);
+    // (bits(t) - bits(1.5 * 2^23)) << 23 == bits(t) << 23 modulo 2^32
+    return make_float2(__uint_as_float(__float_as_uint(pp.x) + (__float_as_uint(tt.x) << 23)),
+                       __uint_as_float(__float_as_uint(pp.y) + (__float_as_uint(tt.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

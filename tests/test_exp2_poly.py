@@ -1,5 +1,5 @@
 """The software base-2 exponential used beside MUFU.EX2 in the tensor-core
-backward: the committed header matches what its generator produces, and the
+forward: the committed header matches what its generator produces, and the
 fp32 evaluation of the device algorithm stays within the stated relative
 error bound against the mathematical 2^x."""
 import importlib.util
@@ -38,8 +38,9 @@ def test_fp32_evaluation_within_bound():
     gen = _gen()
     coeffs, bound = _header()
     assert bound < 1e-4                 # far below bf16's 2^-9 rounding
-    # the bound covers (-126, 0.5]; at -126 and below the clamp test applies
-    x = np.concatenate([np.linspace(-125.99, 0.5, 1000003), [0.0, -1.0, -0.5, 0.5, -125.5]])
+    # the bound covers (-126, 16]; at -126 and below the clamp test applies
+    x = np.concatenate([np.linspace(-125.99, 16.0, 1000003),
+                        [0.0, -1.0, -0.5, 0.5, -125.5, 7.5, 8.0, 15.99]])
     y = gen.fp32_eval(coeffs, x).astype(np.float64)
     ref = np.exp2(x.astype(np.float32).astype(np.float64))
     rel = np.abs(y / ref - 1.0)
