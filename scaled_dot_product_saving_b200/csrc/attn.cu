@@ -208,12 +208,15 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return ATTN_ERR_CUDA;
-    // One CTA per pair of query tiles (p, num_qt - 1 - p) of one head.
+    // One CTA per pair of adjacent query tiles (2p, 2p + 1) of one head; heads
+    // in groups of about 256 CTAs.
     const int num_qt = (n + attn::fwdtc::kBM - 1) / attn::fwdtc::kBM;
-    const long long grid = static_cast<long long>((num_qt + 1) / 2) * BH;
+    const int num_pairs = (num_qt + 1) / 2;
+    const long long grid = static_cast<long long>(num_pairs) * BH;
+    const int head_group = std::max(1, std::min(BH, 256 / num_pairs));
     return traced(ATTN_KERNEL_FWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mo, LSE, n, m, causal, scale * kLog2e, kWaitBudgetNs);
+            mq, mk, mv, mo, LSE, n, m, BH, head_group, causal, scale * kLog2e, kWaitBudgetNs);
         return launched();
     });
 }

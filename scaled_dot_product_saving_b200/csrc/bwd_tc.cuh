@@ -486,7 +486,6 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // 32-column segment at a time, in the 128-byte swizzled layout of the
         // accumulator's tensor map, and one lane hands each segment to the
         // TMA engine as a tiled reduce-add; rows past n are clipped by the TMA.
-        const int r = threadIdx.x - 32 * kWarpDq;
         const int wq = warp & 3;
         const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
         uint8_t* stage = smem + C::kOffdS + wq * C::kStageWarpBytes;

@@ -5,10 +5,11 @@
 // Pass (dQ, dK, dV)", section on the forward; under the causal mask key j > i
 // is excluded before the softmax).
 //
-// One CTA computes two 128-row query tiles, A and B, of one (batch, head),
-// sharing every key and value tile it loads. Query tiles are paired zig-zag
-// (tile p with tile num_qt - 1 - p), so under the causal mask every CTA walks
-// the same number of key tiles. For each 128-key tile t and each query tile x:
+// One CTA computes two adjacent 128-row query tiles, A = 2p and B = 2p + 1,
+// of one (batch, head), sharing every key and value tile it loads; under the
+// causal mask B needs one key tile more than A. CTAs run in groups of heads
+// (so a group's keys and values stay in L2), heaviest query rows first within
+// a group. For each 128-key tile t and each query tile x:
 //   S_x = Q_x K_t^T          tcgen05.mma, both operands K-major in shared
 //                            memory, fp32 accumulator in TMEM
 //   P_x = 2^(S_x * scale * log2e - m_x)   one softmax warpgroup per query
@@ -18,18 +19,20 @@
 //                            written over the S_x columns it came from),
 //                            B = V_t (MN-major), O_x in TMEM
 // The MMA thread issues PV_A(t), S_A(t+1), PV_B(t), S_B(t+1), ... so that the
-// tensor cores work on one tile while the other tile's softmax runs. Because
+// tensor cores work on one tile while the other tile's softmax runs. The
+// softmax hands P over in two halves of 64 keys, and the first half of PV
+// starts while the second half of P is computed. Because
 // S_x(t+1) is issued after PV_x(t) by the same thread, the barrier that reports
 // S_x(t+1) also reports PV_x(t) complete: the softmax may rescale O_x as soon as
 // it sees S_x(t+1).
 //
 // The running maximum is raised, and O rescaled, only when a tile's row
 // maximum exceeds the one in use by more than 2^8 in P, so P <= 256 and the
-// row sum stays well inside fp32. A share of the exponentials is computed on
-// the FMA pipe (exp2_fma_x2) to relieve the MUFU unit; the scaled scores and
-// the row sums use the paired fp32 instructions. At the end O / sum is stored
-// as bf16 through shared memory with the TMA, and the row's natural-log LSE as
-// fp32.
+// row sum stays well inside fp32. The exponentials run on the MUFU unit (a
+// polynomial on the FMA pipe costs more per element on this part than MUFU.EX2
+// does); the scaled scores and the row sums use the paired fp32 instructions,
+// which halve their issue slots. At the end O / sum is stored as bf16 through
+// shared memory with the TMA, and the row's natural-log LSE as fp32.
 //
 // Warp roles (320 threads): warps 0-3 softmax of tile A, warps 4-7 softmax of
 // tile B (warp w reads TMEM lanes 32(w%4) .. 32(w%4)+31), warp 8 TMA producer,
@@ -52,8 +55,6 @@ constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Pairs of a 32-key chunk (bit e = pair e) whose exponentials use the FMA pipe.
-constexpr uint32_t kPolyPairs = 0x8888u;
 
 template <int D>
 struct Cfg {
@@ -81,18 +82,30 @@ struct Bars {
     uint64_t v_full[4];
     uint64_t v_empty[4];
     uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t p_half[2];   // P of keys 0..63 of the tile written
+    uint64_t p_full[2];   // all of P written
     uint64_t o_done[2];
     uint64_t mma_drain;
     uint32_t tmem_base;
     int abort;
 };
 
+// CTA -> (head, pair of query tiles). Heads go in groups of `hg`; within a
+// group the pairs are taken from the last (most key tiles under the causal
+// mask) to the first, each across the group's heads.
+__device__ __forceinline__ void cta_pair(int b, int num_pairs, int BH, int hg, int& bh, int& pair) {
+    const int group = b / (hg * num_pairs);
+    const int within = b % (hg * num_pairs);
+    const int heads_here = min(hg, BH - group * hg);
+    pair = num_pairs - 1 - within / heads_here;
+    bh = group * hg + within % heads_here;
+}
+
 // Maximum (or, for a negative scale, minimum) of a 32-key chunk of raw scores,
-// excluding keys after `kmax` when MASKED.
+// excluding keys after `kmax` when MASKED; two independent chains.
 template <bool NEG, bool MASKED>
-__device__ __forceinline__ float chunk_extreme(const uint32_t (&r)[32], float acc, int key0,
-                                               int kmax) {
+__device__ __forceinline__ float chunk_extreme(const uint32_t (&r)[32], int key0, int kmax) {
+    float acc[2] = {NEG ? INFINITY : -INFINITY, NEG ? INFINITY : -INFINITY};
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
         float a = __uint_as_float(r[e]), b = __uint_as_float(r[e + 1]);
@@ -100,32 +113,29 @@ __device__ __forceinline__ float chunk_extreme(const uint32_t (&r)[32], float ac
             if (key0 + e > kmax) a = NEG ? INFINITY : -INFINITY;
             if (key0 + e + 1 > kmax) b = NEG ? INFINITY : -INFINITY;
         }
-        acc = NEG ? fmin3(acc, a, b) : fmax3(acc, a, b);
+        const int j = (e >> 1) & 1;
+        acc[j] = NEG ? fmin3(acc[j], a, b) : fmax3(acc[j], a, b);
     }
-    return acc;
+    return NEG ? fminf(acc[0], acc[1]) : fmaxf(acc[0], acc[1]);
 }
 
 // P for a 32-key chunk: 2^(raw * scale_log2 - m) (exactly 0 for masked keys),
-// packed to bf16 pairs in `pk`, summed into `sum`.
+// packed to bf16 pairs in `pk`, summed into `sum` (two chains).
 template <bool MASKED>
 __device__ __forceinline__ void chunk_p(const uint32_t (&r)[32], f32x2 sl2, f32x2 neg_m,
-                                        int key0, int kmax, f32x2& sum, uint32_t (&pk)[16]) {
+                                        int key0, int kmax, f32x2 (&sum)[2], uint32_t (&pk)[16]) {
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
         const float2 x = split_f32x2(
             fma_x2(make_f32x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), sl2, neg_m));
         float2 p;
-        if ((kPolyPairs >> e) & 1u) {
-            p = exp2_fma_x2(x.x, x.y);
-        } else {
-            p.x = ex2(x.x);
-            p.y = ex2(x.y);
-        }
+        p.x = ex2(x.x);
+        p.y = ex2(x.y);
         if (MASKED) {
             if (key0 + 2 * e > kmax) p.x = 0.f;
             if (key0 + 2 * e + 1 > kmax) p.y = 0.f;
         }
-        sum = add_x2(sum, make_f32x2(p.x, p.y));
+        sum[e & 1] = add_x2(sum[e & 1], make_f32x2(p.x, p.y));
         pk[e] = pack_bf16x2(p.x, p.y);
     }
 }
@@ -134,8 +144,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-           float* __restrict__ LSE, int n, int m, int causal, float scale_log2,
-           unsigned long long budget_ns) {
+           float* __restrict__ LSE, int n, int m, int BH, int head_group, int causal,
+           float scale_log2, unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
@@ -144,12 +154,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_qt = (n + kBM - 1) / kBM;
     const int num_pairs = (num_qt + 1) / 2;
-    const int bh = int(blockIdx.x) / num_pairs;   // CTAs of one head run together: K/V stay in L2
-    const int pair = int(blockIdx.x) % num_pairs;
+    int bh, pair;
+    cta_pair(int(blockIdx.x), num_pairs, BH, head_group, bh, pair);
     const int num_kt = (m + kBN - 1) / kBN;
-    const bool has_b = num_qt - 1 - pair != pair;
+    const bool has_b = 2 * pair + 1 < num_qt;
     // query tile and number of key tiles of tile A (x = 0) and tile B (x = 1)
-    const int qt_a = pair, qt_b = num_qt - 1 - pair;
+    const int qt_a = 2 * pair, qt_b = 2 * pair + 1;
     const int nkv_a = causal ? min(num_kt, qt_a + 1) : num_kt;
     const int nkv_b = has_b ? (causal ? min(num_kt, qt_b + 1) : num_kt) : 0;
     auto qt_of = [&](int x) { return x ? qt_b : qt_a; };
@@ -171,6 +181,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(&bars->s_full[x], 1);
+            mbar_init(&bars->p_half[x], 128);
             mbar_init(&bars->p_full[x], 128);
             mbar_init(&bars->o_done[x], 1);
         }
@@ -245,12 +256,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
             mma_commit(&bars->s_full[x]);
         };
-        auto issue_PV = [&](int x, int t) {
+        // O_x += P_x V_t over keys 64h .. 64h+63 of the tile
+        auto issue_PV = [&](int x, int t, int h) {
             const uint32_t sV = smem_addr(smem + C::kOffV + (t % C::kVStages) * C::kTileBytes);
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
+            for (int k4 = 0; k4 < 4; ++k4) {
+                const int kk = 4 * h + k4;
                 mma_ts(tmem + C::kColO0 + D * x, tmem + C::kColS0 + 128 * x + kk * 8,
                        sdesc_sw128(sV + kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0));
+            }
         };
         bool ok = mbar_wait(&bars->q_full, 0, abort_flag, budget_ns) &&
                   mbar_wait(&bars->k_full[0], 0, abort_flag, budget_ns);
@@ -264,7 +278,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             bool v_ready = false, k_ready = false;
             for (int x = 0; x < 2; ++x) {
                 if (t >= nkv_of(x)) continue;
-                if (!mbar_wait(&bars->p_full[x], t & 1, abort_flag, budget_ns)) {
+                if (!mbar_wait(&bars->p_half[x], t & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -277,7 +291,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     v_ready = true;
                 }
                 tc_fence_after();
-                issue_PV(x, t);
+                issue_PV(x, t, 0);
+                if (!mbar_wait(&bars->p_full[x], t & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                issue_PV(x, t, 1);
                 if (t + 1 < nkv_of(x)) {
                     if (!k_ready) {
                         const int t1 = t + 1;
@@ -329,25 +349,44 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int k0 = t * kBN;
             const bool masked = __any_sync(0xffffffffu, k0 + kBN - 1 > kmax);
             // pass 1: extreme raw score of the row over this key tile
-            float ext = neg ? INFINITY : -INFINITY;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t ra[32], rb[32];
-                tmem_ld32(tS + 64 * h, ra);
-                tmem_ld32(tS + 64 * h + 32, rb);
-                tmem_ld_wait(ra);
-                tmem_ld_wait(rb);
-                const int key0 = k0 + 64 * h;
+            float ext;
+            {
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tmem_ld32(tS, r0);
+                tmem_ld32(tS + 32, r1);
+                tmem_ld32(tS + 64, r2);
+                tmem_ld32(tS + 96, r3);
+                tmem_ld_wait(r0);
+                tmem_ld_wait(r1);
+                tmem_ld_wait(r2);
+                tmem_ld_wait(r3);
+                float e[4];
                 if (neg) {
-                    ext = masked ? chunk_extreme<true, true>(ra, ext, key0, kmax)
-                                 : chunk_extreme<true, false>(ra, ext, key0, kmax);
-                    ext = masked ? chunk_extreme<true, true>(rb, ext, key0 + 32, kmax)
-                                 : chunk_extreme<true, false>(rb, ext, key0 + 32, kmax);
+                    if (masked) {
+                        e[0] = chunk_extreme<true, true>(r0, k0, kmax);
+                        e[1] = chunk_extreme<true, true>(r1, k0 + 32, kmax);
+                        e[2] = chunk_extreme<true, true>(r2, k0 + 64, kmax);
+                        e[3] = chunk_extreme<true, true>(r3, k0 + 96, kmax);
+                    } else {
+                        e[0] = chunk_extreme<true, false>(r0, k0, kmax);
+                        e[1] = chunk_extreme<true, false>(r1, k0 + 32, kmax);
+                        e[2] = chunk_extreme<true, false>(r2, k0 + 64, kmax);
+                        e[3] = chunk_extreme<true, false>(r3, k0 + 96, kmax);
+                    }
+                    ext = fminf(fminf(e[0], e[1]), fminf(e[2], e[3]));
                 } else {
-                    ext = masked ? chunk_extreme<false, true>(ra, ext, key0, kmax)
-                                 : chunk_extreme<false, false>(ra, ext, key0, kmax);
-                    ext = masked ? chunk_extreme<false, true>(rb, ext, key0 + 32, kmax)
-                                 : chunk_extreme<false, false>(rb, ext, key0 + 32, kmax);
+                    if (masked) {
+                        e[0] = chunk_extreme<false, true>(r0, k0, kmax);
+                        e[1] = chunk_extreme<false, true>(r1, k0 + 32, kmax);
+                        e[2] = chunk_extreme<false, true>(r2, k0 + 64, kmax);
+                        e[3] = chunk_extreme<false, true>(r3, k0 + 96, kmax);
+                    } else {
+                        e[0] = chunk_extreme<false, false>(r0, k0, kmax);
+                        e[1] = chunk_extreme<false, false>(r1, k0 + 32, kmax);
+                        e[2] = chunk_extreme<false, false>(r2, k0 + 64, kmax);
+                        e[3] = chunk_extreme<false, false>(r3, k0 + 96, kmax);
+                    }
+                    ext = fmaxf(fmaxf(e[0], e[1]), fmaxf(e[2], e[3]));
                 }
             }
             const float m_new = fmaxf(m_run, ext * scale_log2);
@@ -375,7 +414,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // pass 2: P as bf16 over the S columns already read (chunk c's P
             // goes to columns 16c .. 16c+15, all read by then)
             const f32x2 neg_m = make_f32x2(-m_run, -m_run);
-            f32x2 sum = make_f32x2(0.f, 0.f);
+            f32x2 sum[2] = {make_f32x2(0.f, 0.f), make_f32x2(0.f, 0.f)};
             uint32_t ra[32], rb[32];
             tmem_ld32(tS, ra);
 #pragma unroll
@@ -390,8 +429,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 else
                     chunk_p<false>(cur, sl2, neg_m, k0 + 32 * c, kmax, sum, pk);
                 tmem_st16(tS + 16 * c, pk);
+                if (c == 1) {
+                    // keys 0..63 of P are in place: the first half of PV may start
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&bars->p_half[x]);
+                }
             }
-            const float2 s2 = split_f32x2(sum);
+            const float2 s2 = split_f32x2(add_x2(sum[0], sum[1]));
             l_run += s2.x + s2.y;
             tmem_st_wait();
             tc_fence_before();

@@ -11,8 +11,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include "exp2_poly.h"
-
 namespace attn {
 
 // Device error word (one per device); written by kernels that give up a wait.
@@ -406,31 +404,6 @@ __device__ __forceinline__ f32x2 add_x2(f32x2 a, f32x2 b) {
     f32x2 r;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
     return r;
-}
-
-// Base-2 exponential of a pair on the FMA pipe, to share the work of the MUFU
-// unit: Cody-Waite reduction 2^x = 2^n * 2^f with n = round(x) (adding and
-// subtracting 1.5 * 2^23 rounds to an integer) and f in [-1/2, 1/2], 2^f from
-// the minimax polynomial of exp2_poly.h (Horner, paired fused multiply-adds),
-// and n added to the result's exponent field. Relative error at most
-// exp2poly::kMaxRelError (7.5e-5) for x in (-126, 16]; inputs at or below -126
-// are clamped there and give a value no larger than 2^-125 rather than 0 --
-// callers that need an exact zero (masked scores) set it themselves.
-__device__ __forceinline__ float2 exp2_fma_x2(float x0, float x1) {
-    const f32x2 x = make_f32x2(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
-    const f32x2 magic = make_f32x2(12582912.0f, 12582912.0f);
-    const f32x2 neg_magic = make_f32x2(-12582912.0f, -12582912.0f);
-    const f32x2 minus1 = make_f32x2(-1.0f, -1.0f);
-    const f32x2 t = add_x2(x, magic);
-    const f32x2 f = fma_x2(add_x2(t, neg_magic), minus1, x);
-    f32x2 p = fma_x2(make_f32x2(exp2poly::kC3, exp2poly::kC3), f,
-                     make_f32x2(exp2poly::kC2, exp2poly::kC2));
-    p = fma_x2(p, f, make_f32x2(exp2poly::kC1, exp2poly::kC1));
-    p = fma_x2(p, f, make_f32x2(exp2poly::kC0, exp2poly::kC0));
-    const float2 pp = split_f32x2(p), tt = split_f32x2(t);
-    // (bits(t) - bits(1.5 * 2^23)) << 23 == bits(t) << 23 modulo 2^32
-    return make_float2(__uint_as_float(__float_as_uint(pp.x) + (__float_as_uint(tt.x) << 23)),
-                       __uint_as_float(__float_as_uint(pp.y) + (__float_as_uint(tt.y) << 23)));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
