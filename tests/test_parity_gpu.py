@@ -69,6 +69,35 @@ def test_cuda_core_path_bf16(d, causal):
     _assert_within(full_compare(w), TOL["bf16"], w.name)
 
 
+@pytest.mark.parametrize("d,causal,scale", [
+    (128, True, -0.09),    # negative scale: the softmax keeps the smallest raw score
+    (64, False, -0.3),
+    (128, False, 0.0),     # zero scale: uniform weights, dQ = dK = 0
+    (64, True, 0.35),      # scale above 1/sqrt(d)
+])
+def test_scale_values(d, causal, scale):
+    """Scales other than 1/sqrt(d) through the tensor-core path."""
+    import numpy as np
+    import oracle.ref as ref
+    from parity_util import rel_err, to64
+    w = synth.make_small(1, 2, 300, 300, d, d, "bf16", causal, seed=77 + d)
+    q, k, v, do = synth.make_inputs(w)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = lib.attn_fwd(qd, kd, vd, causal=causal, scale=scale)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, dod, lse, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert lib.attn_get_device_error() == 0
+    Q, K, V, dO = (t.to(torch.float64).numpy() for t in (q, k, v, do))
+    O_r, lse_r = ref.attention_forward(Q, K, V, causal, scale)
+    dQ_r, dK_r, dV_r = ref.attention_backward(Q, K, V, dO, causal, scale)
+    errs = {name: rel_err(to64(g), r) for name, g, r in
+            zip(("O", "LSE", "dQ", "dK", "dV"), (o, lse, dq, dk, dv), (O_r, lse_r, dQ_r, dK_r, dV_r))}
+    if scale == 0.0:
+        assert np.max(np.abs(dQ_r)) == 0.0 and np.max(np.abs(dK_r)) == 0.0
+    _assert_within(errs, TOL["bf16"], f"d={d} causal={causal} scale={scale}")
+
+
 def test_tensor_path_is_taken():
     lib.attn_set_path(lib.ATTN_PATH_TENSOR)
     w = synth.make_small(1, 1, 256, 256, 64, 64, "bf16", True, seed=3)
