@@ -82,7 +82,9 @@ attn_status_t attn_fwd(const void* Q, const void* K, const void* V,
 /*
  * attn_bwd_workspace_size -- bytes of device scratch that attn_bwd needs for
  * these sizes: D = rowsum(dO * O) and the LSE in base 2, both [B,H,n] fp32
- * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ.
+ * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ
+ * and 256 bytes for the work-item counter of the persistent tensor-core
+ * backward (each region rounded up to 256 bytes).
  * Returns 0 if the sizes are invalid.
  */
 size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv,

@@ -57,7 +57,7 @@ attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, bool* use_tensor) {
 }
 
 struct Workspace {
-    size_t lse2_off, dd_off, dq_off, total;
+    size_t lse2_off, dd_off, dq_off, sched_off, total;
     int n_pad;
 };
 
@@ -69,7 +69,8 @@ Workspace carve(int B, int H, int n, int d) {
     w.lse2_off = 0;
     w.dd_off = row_bytes;
     w.dq_off = 2 * row_bytes;
-    w.total = w.dq_off + round_up(bh * static_cast<size_t>(n) * d * sizeof(float), 256);
+    w.sched_off = w.dq_off + round_up(bh * static_cast<size_t>(n) * d * sizeof(float), 256);
+    w.total = w.sched_off + 256;   // the backward's work-item counter
     return w;
 }
 
@@ -223,8 +224,8 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
 
 template <typename T>
 attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float* lse2, float* Dd,
-                         float* dQacc, int BH, int n, int n_pad, int d, int dv, float d_scale,
-                         cudaStream_t st) {
+                         float* dQacc, int* sched, int BH, int n, int n_pad, int d, int dv,
+                         float d_scale, cudaStream_t st) {
     const size_t rows = static_cast<size_t>(BH) * n_pad;
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
     const bool vec = sizeof(T) == 2 && dv % 8 == 0 && (dv / 8) <= 32 && 32 % (dv / 8) == 0 &&
@@ -235,15 +236,15 @@ attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float*
         return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
             attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
-                lse2, Dd, dQacc, dq_elems, BH, n, n_pad, dv, d_scale);
+                lse2, Dd, dQacc, sched, dq_elems, BH, n, n_pad, dv, d_scale);
             return launched();
         });
     }
     const int grid = grid_for(rows, attn::prep::kThreads / 32, 148 * 16);
     return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
         attn::prep::preprocess_generic<T><<<grid, attn::prep::kThreads, 0, st>>>(
-            static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, dq_elems,
-            BH, n, n_pad, dv, d_scale);
+            static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, sched,
+            dq_elems, BH, n, n_pad, dv, d_scale);
         return launched();
     });
 }
@@ -281,7 +282,7 @@ attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* 
 
 template <int D>
 attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void* dO,
-                         const float* lse2, const float* Dd, int n_pad, float* dQacc, void* dK,
+                         const float* lse2, const float* Dd, int* sched, int n_pad, float* dQacc, void* dK,
                          void* dV, int BH, int n, int m, int causal, float scale,
                          cudaStream_t st) {
     using C = attn::bwdtc::Cfg<D>;
@@ -296,14 +297,16 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
         return ATTN_ERR_CUDA;
+    // Persistent: one CTA per SM (at most one per work item), each walking
+    // the work items (key tile, head) with a stride of the grid size; heads
+    // per scheduling group: about 256 items a group.
     const int num_kt = (m + kTile - 1) / kTile;
-    const long long grid = static_cast<long long>(num_kt) * BH;
-    // heads per scheduling group: about 256 CTAs a group
+    const long long items = static_cast<long long>(num_kt) * BH;
+    const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     const int head_group = std::max(1, std::min(BH, 256 / num_kt));
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, n_pad, n, m, BH, head_group, sm_count(),
-            causal, scale,
+            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, sched, n_pad, n, m, BH, head_group, causal, scale,
             scale * kLog2e, kWaitBudgetNs);
         return launched();
     });
@@ -390,20 +393,22 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
     float* Dd = reinterpret_cast<float*>(ws + w.dd_off);
     float* dQacc = reinterpret_cast<float*>(ws + w.dq_off);
+    int* sched = reinterpret_cast<int*>(ws + w.sched_off);
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
 
     // The tensor-core backward takes D already multiplied by the scale.
     const float d_scale = tensor ? scale : 1.0f;
     s = (dtype == ATTN_F32)
-            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv, d_scale, st)
-            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, BH, n, w.n_pad, d, dv,
+            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv, d_scale,
+                                st)
+            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv,
                                         d_scale, st);
     if (s != ATTN_OK) return s;
     if (tensor) {
-        s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, w.n_pad, dQacc, dK, dV, BH, n, m,
-                                       causal, scale, st)
-                      : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, w.n_pad, dQacc, dK, dV, BH, n, m,
-                                        causal, scale, st);
+        s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
+                                       n, m, causal, scale, st)
+                      : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
+                                        n, m, causal, scale, st);
         if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, 1.0f, st);
     } else if (dtype == ATTN_F32) {
         s = bwd_simt<float>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv, causal,

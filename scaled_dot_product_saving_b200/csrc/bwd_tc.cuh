@@ -78,7 +78,7 @@ struct Cfg {
     static constexpr int kOffLse = kOffdS + 128 * 128 * 2;
     static constexpr int kOffDd = kOffLse + kStages * kBM * 4;
     static constexpr int kOffBar = kOffDd + kStages * kBM * 4;
-    static constexpr int kSmemBytes = kOffBar + 256;
+    static constexpr int kSmemBytes = kOffBar + 512;
     static constexpr bool kAlias = (D == 128);
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColdV = 0;
@@ -96,6 +96,7 @@ struct Cfg {
 
 struct Bars {
     uint64_t kv_full;
+    uint64_t kv_empty;      // the item's last MMA has read K_j, V_j
     uint64_t q_full[4];
     uint64_t q_empty[4];
     uint64_t s_full;
@@ -105,10 +106,16 @@ struct Bars {
     uint64_t ds_smem_full;
     uint64_t ds_smem_free;
     uint64_t acc_done;
+    uint64_t acc_free;      // the epilogue has read dV, dK out of TMEM
+    uint64_t epi_done[4];   // an item's dV, dK staged in stage s and read by the TMA
     uint64_t mma_drain;
+    uint64_t sched_full[4];     // work item of slot k published by the producer
+    uint64_t sched_empty[4];    // ... and read by the 13 consumers
+    int sched_item[4];
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Bars) <= 512, "barrier area");
 
 // Sixteen queries (columns q0..q0+15 of a tile) for one key row: P^T and dS^T
 // from the S^T / dP^T values in registers. P^T and dS^T are written back to
@@ -158,7 +165,8 @@ __device__ __forceinline__ void store_ds_chunk(uint8_t* sdS, int c, int r, const
     }
 }
 
-// The (head, key tile) of CTA `b` in launch order (see the kernel's comment).
+// The (head, key tile) of work item `b` in schedule order (see the kernel's
+// comment).
 __device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int& bh, int& kt) {
     const int group = b / (hg * num_kt);
     const int within = b % (hg * num_kt);
@@ -167,14 +175,28 @@ __device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int&
     bh = group * hg + within % heads_here;
 }
 
+// One work item: 128 keys of one head and the query tiles that see them.
+struct Item {
+    int bh, k0, first_qt, T;
+};
+__device__ __forceinline__ Item item_at(int b, int num_kt, int num_qt, int BH, int hg, int causal) {
+    Item it;
+    int kt;
+    cta_tile(b, num_kt, BH, hg, it.bh, kt);
+    it.k0 = kt * kBN;
+    it.first_qt = causal ? kt : 0;
+    it.T = num_qt - it.first_qt;          // >= 1
+    return it;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
            const __grid_constant__ CUtensorMap tmdQacc, const __grid_constant__ CUtensorMap tmdK,
-           const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ lse2, const float* __restrict__ Dd, int n_pad,
-           int n, int m, int BH, int head_group,
-           int prefetch_stride, int causal, float scale, float scale_log2,
+           const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ lse2,
+           const float* __restrict__ Dd, int* __restrict__ sched, int n_pad, int n, int m, int BH,
+           int head_group, int causal, float scale, float scale_log2,
            unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -182,17 +204,34 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     volatile int* abort_flag = &bars->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // CTA order: heads in groups of `hg` (about 256 CTAs a group, so the
-    // heads in flight keep their Q/dO tiles and dQ rows in L2); inside a group
-    // key-tile major, so the longest CTAs of the group (lowest key tiles, if
-    // causal) start first and the shortest run last.
+    // Persistent: G CTAs (at most one per SM). CTA c starts with work item
+    // c, and takes every further item from a global counter (zeroed by the
+    // preprocess kernel) as it goes, so items are handed out in order to
+    // whichever CTA is ready. Items are ordered in groups of `head_group`
+    // heads (about 256 items a group, so the heads in flight keep their Q/dO
+    // tiles and dQ rows in L2); inside a group key-tile major, so the longest
+    // items of the group (lowest key tiles, if causal) come first. The
+    // producer publishes each item to the other roles through a 4-slot ring
+    // in shared memory, one item ahead.
     const int num_kt = (m + kBN - 1) / kBN;
-    int bh, kt;
-    cta_tile(int(blockIdx.x), num_kt, BH, head_group, bh, kt);
-    const int k0 = kt * kBN;
     const int num_qt = (n + kBM - 1) / kBM;
-    const int first_qt = causal ? kt : 0;
-    const int T = num_qt - first_qt;          // query tiles this CTA visits (>= 1)
+    const int num_items = num_kt * BH;
+    const int G = int(gridDim.x);
+    auto item = [&](int b) { return item_at(b, num_kt, num_qt, BH, head_group, causal); };
+    // Consumers: the work item of the j-th slot (-1 = no more), or -2 if
+    // the wait gave up. A warp reads it in every lane, then lane 0 releases
+    // the slot; the MMA thread passes warp = false.
+    auto next_item = [&](int j, bool warp_wide) -> int {
+        const int slot = j & 3;
+        const bool got = warp_wide
+                             ? mbar_wait_warp(&bars->sched_full[slot], (j >> 2) & 1, abort_flag, budget_ns)
+                             : mbar_wait(&bars->sched_full[slot], (j >> 2) & 1, abort_flag, budget_ns);
+        if (!got) return -2;
+        const int b = *reinterpret_cast<volatile int*>(&bars->sched_item[slot]);
+        if (warp_wide) __syncwarp();
+        if (!warp_wide || (threadIdx.x & 31) == 0) mbar_arrive(&bars->sched_empty[slot]);
+        return b;
+    };
 
     if (threadIdx.x == 0) {
         // The swizzled tiles need a 1024-byte aligned base. A CTA that starts
@@ -201,6 +240,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         if (misaligned) record_device_error(kErrTimeout);
         bars->abort = (misaligned || *reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0) ? 1 : 0;
         mbar_init(&bars->kv_full, 1);
+        mbar_init(&bars->kv_empty, 1);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
@@ -212,7 +252,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         mbar_init(&bars->ds_smem_full, 256);
         mbar_init(&bars->ds_smem_free, 128);
         mbar_init(&bars->acc_done, 1);
+        mbar_init(&bars->acc_free, 256);
+        for (int s = 0; s < 4; ++s) mbar_init(&bars->epi_done[s], 256);
         mbar_init(&bars->mma_drain, 1);
+        for (int k = 0; k < 4; ++k) {
+            mbar_init(&bars->sched_full[k], 1);
+            mbar_init(&bars->sched_empty[k], 1 + 8 + 4);
+        }
         fence_mbar_init();
     }
     if (warp == kWarpMma) {
@@ -223,7 +269,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const bool aborted_early = bars->abort != 0 || T <= 0;
+    const bool aborted_early = bars->abort != 0;
 
     if (!aborted_early && warp == kWarpProducer && lane == 0) {
         // ------------------------------------------------ TMA producer
@@ -234,46 +280,93 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         prefetch_tensor_map(&tmdQacc);
         prefetch_tensor_map(&tmdK);
         prefetch_tensor_map(&tmdV);
-        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
-        for (int p = 0; p < C::kPanels; ++p) {
-            tma_load_3d(smem + C::kOffK + p * C::kPanelBytes, &tmK, &bars->kv_full, p * 64, k0, bh);
-            tma_load_3d(smem + C::kOffV + p * C::kPanelBytes, &tmV, &bars->kv_full, p * 64, k0, bh);
-        }
-        // Warm L2 with the K/V tiles of the CTA that will most likely start on
-        // a free SM about one CTA lifetime from now.
-        if (int(blockIdx.x) + prefetch_stride < int(gridDim.x)) {
-            int nbh, nkt;
-            cta_tile(int(blockIdx.x) + prefetch_stride, num_kt, BH, head_group, nbh, nkt);
-            for (int p = 0; p < C::kPanels; ++p) {
-                tma_prefetch_l2_3d(&tmK, p * 64, nkt * kBN, nbh);
-                tma_prefetch_l2_3d(&tmV, p * 64, nkt * kBN, nbh);
+        // Q_i, dO_i and the LSE/D slices of one query tile into stage g % S
+        // (g counts query tiles over all of this CTA's items). A stage that
+        // held an item's last tile also holds that item's dV/dK epilogue
+        // staging: it is reloaded once the epilogue is done with it.
+        uint32_t last_in = 0;      // bit s: stage s held an item's last tile
+        uint32_t epi_parity = 0;   // bit s: parity of the next epi_done[s] phase
+        auto load_q = [&](const Item& it, int t, int g) -> bool {
+            const int s = g % C::kStages;
+            const int q0 = (it.first_qt + t) * kBM;
+            if (g >= C::kStages &&
+                !mbar_wait(&bars->q_empty[s], (g / C::kStages - 1) & 1, abort_flag, budget_ns))
+                return false;
+            if ((last_in >> s) & 1u) {
+                if (!mbar_wait(&bars->epi_done[s], (epi_parity >> s) & 1u, abort_flag, budget_ns))
+                    return false;
+                epi_parity ^= 1u << s;
             }
-        }
-        int issued = 0;
-        for (int t = 0; t < T; ++t) {
-            const int s = t % C::kStages, k = t / C::kStages;
-            const int q0 = (first_qt + t) * kBM;
-            if (t >= C::kStages &&
-                !mbar_wait(&bars->q_empty[s], (k - 1) & 1, abort_flag, budget_ns)) {
-                record_device_error(kErrTimeout);
-                *abort_flag = 1;
-                break;
-            }
+            last_in = (last_in & ~(1u << s)) | (uint32_t(t == it.T - 1) << s);
             mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::kTileBytes + 2 * kBM * 4);
             for (int p = 0; p < C::kPanels; ++p) {
                 tma_load_3d(smem + C::kOffQ + s * C::kTileBytes + p * C::kPanelBytes, &tmQ,
-                            &bars->q_full[s], p * 64, q0, bh);
+                            &bars->q_full[s], p * 64, q0, it.bh);
                 tma_load_3d(smem + C::kOffdO + s * C::kTileBytes + p * C::kPanelBytes, &tmdO,
-                            &bars->q_full[s], p * 64, q0, bh);
+                            &bars->q_full[s], p * 64, q0, it.bh);
             }
-            bulk_load(smem + C::kOffLse + s * kBM * 4, lse2 + size_t(bh) * n_pad + q0, kBM * 4,
+            bulk_load(smem + C::kOffLse + s * kBM * 4, lse2 + size_t(it.bh) * n_pad + q0, kBM * 4,
                       &bars->q_full[s]);
-            bulk_load(smem + C::kOffDd + s * kBM * 4, Dd + size_t(bh) * n_pad + q0, kBM * 4,
+            bulk_load(smem + C::kOffDd + s * kBM * 4, Dd + size_t(it.bh) * n_pad + q0, kBM * 4,
                       &bars->q_full[s]);
-            ++issued;
+            return true;
+        };
+        auto publish = [&](int k, int b) -> bool {
+            const int slot = k & 3;
+            if (k >= 4 &&
+                !mbar_wait(&bars->sched_empty[slot], ((k >> 2) - 1) & 1, abort_flag, budget_ns))
+                return false;
+            bars->sched_item[slot] = b;
+            mbar_arrive(&bars->sched_full[slot]);
+            return true;
+        };
+        int g = 0, kv_issued = 0;
+        int b = int(blockIdx.x);
+        bool ok = publish(0, b);
+        for (int j = 0; ok; ++j) {
+            const Item it = item(b);
+            // The first query tile goes in as soon as a stage is free; K_j and
+            // V_j once the previous item's last MMA has read its own.
+            if (!load_q(it, 0, g)) { ok = false; break; }
+            ++g;
+            if (j > 0 && !mbar_wait(&bars->kv_empty, (j - 1) & 1, abort_flag, budget_ns)) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+            for (int p = 0; p < C::kPanels; ++p) {
+                tma_load_3d(smem + C::kOffK + p * C::kPanelBytes, &tmK, &bars->kv_full, p * 64, it.k0, it.bh);
+                tma_load_3d(smem + C::kOffV + p * C::kPanelBytes, &tmV, &bars->kv_full, p * 64, it.k0, it.bh);
+            }
+            ++kv_issued;
+            for (int t = 1; t < it.T; ++t) {
+                if (!load_q(it, t, g)) { ok = false; break; }
+                ++g;
+            }
+            if (!ok) break;
+            // All of this item's loads are issued (a couple of tiles ahead of
+            // the MMAs): take the next item now, publish it, and warm L2 with
+            // its K/V.
+            int nb = G + atomicAdd(sched, 1);
+            if (nb >= num_items) nb = -1;
+            if (!publish(j + 1, nb)) { ok = false; break; }
+            if (nb < 0) break;
+            const Item nx = item(nb);
+            for (int p = 0; p < C::kPanels; ++p) {
+                tma_prefetch_l2_3d(&tmK, p * 64, nx.k0, nx.bh);
+                tma_prefetch_l2_3d(&tmV, p * 64, nx.k0, nx.bh);
+            }
+            b = nb;
         }
-        (void)mbar_wait_timed(&bars->kv_full, 0, budget_ns);
-        for (int t = (issued > C::kStages ? issued - C::kStages : 0); t < issued; ++t)
+        if (!ok) {
+            record_device_error(kErrTimeout);
+            *abort_flag = 1;
+        }
+        // Drain: every load issued must land before the CTA may exit. Loads
+        // older than the last stage's worth (and K/V before the last) were
+        // consumed, so they have landed.
+        if (kv_issued > 0) (void)mbar_wait_timed(&bars->kv_full, (kv_issued - 1) & 1, budget_ns);
+        for (int t = (g > C::kStages ? g - C::kStages : 0); t < g; ++t)
             (void)mbar_wait_timed(&bars->q_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
     } else if (!aborted_early && warp == kWarpMma && lane == 0) {
         // ------------------------------------------------ MMA issuer
@@ -283,77 +376,98 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sK = smem_addr(smem + C::kOffK);
         const uint32_t sV = smem_addr(smem + C::kOffV);
         const uint32_t sdS = smem_addr(smem + C::kOffdS);
-        bool ok = mbar_wait(&bars->kv_full, 0, abort_flag, budget_ns);
-        for (int t = 0; ok && t < T; ++t) {
-            const int s = t % C::kStages;
-            const uint32_t sQ = smem_addr(smem + C::kOffQ + s * C::kTileBytes);
-            const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
-            if (!mbar_wait(&bars->q_full[s], (t / C::kStages) & 1, abort_flag, budget_ns)) {
+        bool ok = true;
+        int g = 0;
+        for (int j = 0; ok; ++j) {
+            const int b = next_item(j, false);
+            if (b == -1) break;
+            if (b < 0) { ok = false; break; }
+            const int T = item(b).T;
+            if (!mbar_wait(&bars->kv_full, j & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
-            tc_fence_after();
-            // dP^T first: its columns are free once the previous dK MMAs
-            // (issued earlier) have read dS^T from them.
+            for (int t = 0; t < T; ++t, ++g) {
+                const int s = g % C::kStages;
+                const uint32_t sQ = smem_addr(smem + C::kOffQ + s * C::kTileBytes);
+                const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
+                if (!mbar_wait(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                // dP^T first: its columns are free once the previous dK MMAs
+                // (issued earlier) have read dS^T from them.
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
-            }
-            // S^T shares its columns with the previous tile's dQ (d = 128).
-            if (C::kAlias && t > 0 &&
-                !mbar_wait(&bars->dq_free, (t - 1) & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
-                       sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
-            }
-            mma_commit(&bars->s_full);
-            // dV += P^T dO and dK += dS^T Q, 32 queries (two k-steps) per chunk
-            // as soon as a P/dS warpgroup has written that chunk; the two
-            // warpgroups finish chunks 0 and 2 first, then 1 and 3.
-            bool first = (t == 0);
-            for (int ci = 0; ci < kChunks; ++ci) {
-                const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
-                if (!mbar_wait(&bars->ds_chunk[c], t & 1, abort_flag, budget_ns)) {
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                           sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
+                }
+                // S^T shares its columns with the previous tile's dQ (d = 128).
+                if (C::kAlias && g > 0 &&
+                    !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int kk = 2 * c + h;                      // queries 16kk..16kk+15
-                    mma_ts(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
-                           sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
-                    mma_ts(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
-                           sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
-                    first = false;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                    mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
+                           sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
                 }
-            }
-            if (!ok) break;
-            mma_commit(&bars->q_empty[s]);
-            if (t == T - 1) mma_commit(&bars->acc_done);
-            if (!C::kAlias && t > 0 &&
-                !mbar_wait(&bars->dq_free, (t - 1) & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            if (!mbar_wait(&bars->ds_smem_full, t & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
+                mma_commit(&bars->s_full);
+                // The item's first dV/dK MMAs overwrite the accumulators: the
+                // previous item's epilogue must have read them out.
+                if (t == 0 && j > 0 &&
+                    !mbar_wait(&bars->acc_free, (j - 1) & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                // dV += P^T dO and dK += dS^T Q, 32 queries (two k-steps) per
+                // chunk as soon as a P/dS warpgroup has written that chunk; the
+                // two warpgroups finish chunks 0 and 2 first, then 1 and 3.
+                bool first = (t == 0);
+                for (int ci = 0; ci < kChunks; ++ci) {
+                    const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
+                    if (!mbar_wait(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
-                mma_ss(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
-                       sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0);
-            mma_commit(&bars->dq_full);
+                    for (int h = 0; h < 2; ++h) {
+                        const int kk = 2 * c + h;                      // queries 16kk..16kk+15
+                        mma_ts(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
+                               sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                        mma_ts(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
+                               sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                        first = false;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bars->q_empty[s]);
+                if (t == T - 1) mma_commit(&bars->acc_done);
+                if (!C::kAlias && g > 0 &&
+                    !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                if (!mbar_wait(&bars->ds_smem_full, g & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ss(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
+                           sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0);
+                mma_commit(&bars->dq_full);
+                // The item's last MMA has been issued: K_j, V_j are free once
+                // it has completed.
+                if (t == T - 1) mma_commit(&bars->kv_empty);
+            }
         }
         if (!ok) {
             record_device_error(kErrTimeout);
@@ -366,115 +480,139 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int grp = warp >> 2;                       // chunks 2*grp and 2*grp+1
         const int r = threadIdx.x & 127;                 // key row in the tile == TMEM lane
         const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16);
-        const int j = k0 + r;
-        const bool key_ok = j < m;
         uint8_t* sdS = smem + C::kOffdS;
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int s = t % C::kStages;
-            const int q0 = (first_qt + t) * kBM;
-            if (!mbar_wait_warp(&bars->q_full[s], (t / C::kStages) & 1, abort_flag, budget_ns) ||
-                !mbar_wait_warp(&bars->s_full, t & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const float* lse_s = reinterpret_cast<const float*>(smem + C::kOffLse + s * kBM * 4);
-            const float* dd_s = reinterpret_cast<const float*>(smem + C::kOffDd + s * kBM * 4);
-            // Keys past the end get P = 0 in every column; on the diagonal tile,
-            // key r is masked for the queries in the tile before it (q < r).
-            // The masked variant is chosen per warp, never per lane: it holds
-            // warp-collective tcgen05.st instructions, which must not sit in a
-            // divergent branch. Lanes that need no mask get a bound of 0.
-            const bool diag = causal && (q0 == k0);
-            const int below = !key_ok ? kBM : (diag ? r : 0);
-            const bool masked = __any_sync(0xffffffffu, below > 0);
-            // Four half-chunks of 16 queries (two chunks), each half's TMEM
-            // loads issued while the previous half is computed. A chunk's
-            // P^T/dS^T go into the first 16 of its own 32 columns: half h of
-            // chunk c writes columns 32c+8h..32c+8h+7, which it has read.
-            uint32_t ds0[16], ds1[16];
-            uint32_t sA[16], pA[16], sB[16], pB[16];
-            const int cbase = 2 * grp;
-            tmem_ld16(tl + C::kColS + cbase * 32, sA);
-            tmem_ld16(tl + C::kColdP + cbase * 32, pA);
-            tmem_ld_wait();
-#pragma unroll
-            for (int hc = 0; hc < 4; ++hc) {
-                const int c = cbase + (hc >> 1), half = hc & 1;
-                const int qcol = 32 * c + 16 * half;              // first query of the half
-                uint32_t (&scur)[16] = (hc & 1) ? sB : sA;
-                uint32_t (&pcur)[16] = (hc & 1) ? pB : pA;
-                uint32_t (&snxt)[16] = (hc & 1) ? sA : sB;
-                uint32_t (&pnxt)[16] = (hc & 1) ? pA : pB;
-                if (hc < 3) {
-                    const int qn = 32 * (cbase + ((hc + 1) >> 1)) + 16 * ((hc + 1) & 1);
-                    tmem_ld16(tl + C::kColS + qn, snxt);
-                    tmem_ld16(tl + C::kColdP + qn, pnxt);
+        int g = 0;
+        for (int j = 0; ok; ++j) {
+            const int b = next_item(j, true);
+            if (b == -1) break;
+            if (b < 0) { ok = false; break; }
+            const Item it = item(b);
+            const bool key_ok = it.k0 + r < m;
+            for (int t = 0; t < it.T; ++t, ++g) {
+                const int s = g % C::kStages;
+                const int q0 = (it.first_qt + t) * kBM;
+                if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns) ||
+                    !mbar_wait_warp(&bars->s_full, g & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
                 }
-                uint32_t* dk = ((hc >> 1) ? ds1 : ds0) + 8 * half;
-                const uint32_t pcol = tl + C::kColP + 32 * c + 8 * half;
-                const uint32_t dscol = tl + C::kColdS + 32 * c + 8 * half;
-                if (masked)
-                    pds_half<true>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
-                                   dscol, dk);
-                else
-                    pds_half<false>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
-                                    dscol, dk);
-                if (half == 1) {
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(&bars->ds_chunk[c]);
-                }
-                if (hc < 3) tmem_ld_wait();
-            }
-            // The dS tile doubles as the dQ warpgroup's staging buffer for the
-            // previous tile: write it once the TMA engine has read that.
-            if (t > 0 &&
-                !mbar_wait_warp(&bars->ds_smem_free, (t - 1) & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            store_ds_chunk<D>(sdS, 2 * grp, r, ds0);
-            store_ds_chunk<D>(sdS, 2 * grp + 1, r, ds1);
-            fence_proxy_async_smem();
-            mbar_arrive(&bars->ds_smem_full);
-        }
-        // Epilogue: group 0 writes dV, group 1 writes dK. Each warp converts
-        // its 32 rows to bf16 in the 128-byte swizzled layout of the output's
-        // tensor map, staged in this CTA's Q / dO stage buffers (every MMA
-        // that read them is complete once acc_done has fired), and one lane
-        // stores 32 x 64 boxes with the TMA; rows past m are clipped.
-        if (ok && !mbar_wait_warp(&bars->acc_done, 0, abort_flag, budget_ns)) ok = false;
-        if (ok) {
-            tc_fence_after();
-            const uint32_t col = grp == 0 ? C::kColdV : C::kColdK;
-            const CUtensorMap* out_map = grp == 0 ? &tmdV : &tmdK;
-            uint8_t* stage = smem + (grp == 0 ? C::kOffQ : C::kOffdO) + (warp & 3) * (32 * D * 2);
-#pragma unroll
-            for (int pnl = 0; pnl < C::kPanels; ++pnl) {
-                uint32_t rr[64];
-                tmem_ld32(tl + col + 64 * pnl, *reinterpret_cast<uint32_t(*)[32]>(rr));
-                tmem_ld32(tl + col + 64 * pnl + 32, *reinterpret_cast<uint32_t(*)[32]>(rr + 32));
+                tc_fence_after();
+                const float* lse_s = reinterpret_cast<const float*>(smem + C::kOffLse + s * kBM * 4);
+                const float* dd_s = reinterpret_cast<const float*>(smem + C::kOffDd + s * kBM * 4);
+                // Keys past the end get P = 0 in every column; on the diagonal
+                // tile, key r is masked for the queries in the tile before it
+                // (q < r). The masked variant is chosen per warp, never per
+                // lane: it holds warp-collective tcgen05.st instructions, which
+                // must not sit in a divergent branch. Lanes that need no mask
+                // get a bound of 0.
+                const bool diag = causal && (q0 == it.k0);
+                const int below = !key_ok ? kBM : (diag ? r : 0);
+                const bool masked = __any_sync(0xffffffffu, below > 0);
+                // Four half-chunks of 16 queries (two chunks), each half's TMEM
+                // loads issued while the previous half is computed. A chunk's
+                // P^T/dS^T go into the first 16 of its own 32 columns: half h
+                // of chunk c writes columns 32c+8h..32c+8h+7, which it has read.
+                uint32_t ds0[16], ds1[16];
+                uint32_t sA[16], pA[16], sB[16], pB[16];
+                const int cbase = 2 * grp;
+                tmem_ld16(tl + C::kColS + cbase * 32, sA);
+                tmem_ld16(tl + C::kColdP + cbase * 32, pA);
                 tmem_ld_wait();
-                uint8_t* buf = stage + pnl * 4096;
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) = make_uint4(
-                        pack_bf16x2(__uint_as_float(rr[8 * k + 0]), __uint_as_float(rr[8 * k + 1])),
-                        pack_bf16x2(__uint_as_float(rr[8 * k + 2]), __uint_as_float(rr[8 * k + 3])),
-                        pack_bf16x2(__uint_as_float(rr[8 * k + 4]), __uint_as_float(rr[8 * k + 5])),
-                        pack_bf16x2(__uint_as_float(rr[8 * k + 6]), __uint_as_float(rr[8 * k + 7])));
+                for (int hc = 0; hc < 4; ++hc) {
+                    const int c = cbase + (hc >> 1), half = hc & 1;
+                    const int qcol = 32 * c + 16 * half;              // first query of the half
+                    uint32_t (&scur)[16] = (hc & 1) ? sB : sA;
+                    uint32_t (&pcur)[16] = (hc & 1) ? pB : pA;
+                    uint32_t (&snxt)[16] = (hc & 1) ? sA : sB;
+                    uint32_t (&pnxt)[16] = (hc & 1) ? pA : pB;
+                    if (hc < 3) {
+                        const int qn = 32 * (cbase + ((hc + 1) >> 1)) + 16 * ((hc + 1) & 1);
+                        tmem_ld16(tl + C::kColS + qn, snxt);
+                        tmem_ld16(tl + C::kColdP + qn, pnxt);
+                    }
+                    uint32_t* dk = ((hc >> 1) ? ds1 : ds0) + 8 * half;
+                    const uint32_t pcol = tl + C::kColP + 32 * c + 8 * half;
+                    const uint32_t dscol = tl + C::kColdS + 32 * c + 8 * half;
+                    if (masked)
+                        pds_half<true>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
+                                       dscol, dk);
+                    else
+                        pds_half<false>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
+                                        dscol, dk);
+                    if (half == 1) {
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(&bars->ds_chunk[c]);
+                    }
+                    if (hc < 3) tmem_ld_wait();
+                }
+                // The dS tile doubles as the dQ warpgroup's staging buffer for
+                // the previous tile: write it once the TMA has read that.
+                if (g > 0 &&
+                    !mbar_wait_warp(&bars->ds_smem_free, (g - 1) & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
+                }
+                store_ds_chunk<D>(sdS, 2 * grp, r, ds0);
+                store_ds_chunk<D>(sdS, 2 * grp + 1, r, ds1);
+                fence_proxy_async_smem();
+                mbar_arrive(&bars->ds_smem_full);
+            }
+            if (!ok) break;
+            // Epilogue of item j: group 0 writes dV, group 1 writes dK, staged
+            // in the Q / dO halves of the stage that held the item's last tile
+            // (every MMA that read it is complete once acc_done has fired; the
+            // producer reloads it only after epi_done). Each thread reads its
+            // key row out of TMEM 32 columns at a time, converts it to bf16
+            // and stages it in the 128-byte swizzled layout of the output's
+            // tensor map; one lane per warp stores 32 x 64 boxes with the TMA
+            // (rows past m clipped). The accumulators are released for the
+            // next item as soon as they have been read.
+            if (!mbar_wait_warp(&bars->acc_done, j & 1, abort_flag, budget_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {
+                const int s_last = (g - 1) % C::kStages;
+                const uint32_t col = grp == 0 ? C::kColdV : C::kColdK;
+                uint8_t* stage = smem + (grp == 0 ? C::kOffQ : C::kOffdO) + s_last * C::kTileBytes +
+                                 (warp & 3) * (32 * D * 2);
+#pragma unroll
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t rr[32];
+                    tmem_ld32(tl + col + 32 * q, rr);
+                    tmem_ld_wait(rr);
+                    uint8_t* buf = stage + (q >> 1) * 4096;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int kc = 4 * (q & 1) + k;            // 16-byte chunk of the 128-byte row
+                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((kc ^ (lane & 7)) * 16)) = make_uint4(
+                            pack_bf16x2(__uint_as_float(rr[8 * k + 0]), __uint_as_float(rr[8 * k + 1])),
+                            pack_bf16x2(__uint_as_float(rr[8 * k + 2]), __uint_as_float(rr[8 * k + 3])),
+                            pack_bf16x2(__uint_as_float(rr[8 * k + 4]), __uint_as_float(rr[8 * k + 5])),
+                            pack_bf16x2(__uint_as_float(rr[8 * k + 6]), __uint_as_float(rr[8 * k + 7])));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->acc_free);
+                const CUtensorMap* out_map = grp == 0 ? &tmdV : &tmdK;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(out_map, buf, 64 * pnl, k0 + 32 * (warp & 3), bh);
+#pragma unroll
+                    for (int pnl = 0; pnl < C::kPanels; ++pnl)
+                        tma_store_3d(out_map, stage + pnl * 4096, 64 * pnl, it.k0 + 32 * (warp & 3), it.bh);
                     bulk_commit_group();
+                    bulk_wait_group_read0();
                 }
+                __syncwarp();
+                mbar_arrive(&bars->epi_done[s_last]);
             }
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-        } else {
+        }
+        if (!ok) {
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
@@ -490,49 +628,56 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
         uint8_t* stage = smem + C::kOffdS + wq * C::kStageWarpBytes;
         bool ok = true;
-        for (int t = 0; t < T; ++t) {
-            const int row0 = (first_qt + t) * kBM + wq * 32;
-            if (!mbar_wait_warp(&bars->dq_full, t & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            // 64 columns at a time; the TMEM columns are released (dq_free)
-            // as soon as the last of them is in registers.
-#pragma unroll
-            for (int pair = 0; pair < D / 64; ++pair) {
-                uint32_t v[64];
-                tmem_ld32(tl + C::kColdQ + 64 * pair, *reinterpret_cast<uint32_t(*)[32]>(v));
-                tmem_ld32(tl + C::kColdQ + 64 * pair + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                tmem_ld_wait();
-                if (pair == D / 64 - 1) {
-                    tc_fence_before();
-                    mbar_arrive(&bars->dq_free);
+        int g = 0;
+        for (int j = 0; ok; ++j) {
+            const int b = next_item(j, true);
+            if (b == -1) break;
+            if (b < 0) { ok = false; break; }
+            const Item it = item(b);
+            for (int t = 0; t < it.T; ++t, ++g) {
+                const int row0 = (it.first_qt + t) * kBM + wq * 32;
+                if (!mbar_wait_warp(&bars->dq_full, g & 1, abort_flag, budget_ns)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                // 64 columns at a time; the TMEM columns are released (dq_free)
+                // as soon as the last of them is in registers.
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int g = 2 * pair + hh;                  // columns 32g..32g+31
-                    uint8_t* buf = stage + hh * 4096;
-                    if (g >= 2) {
-                        if (lane == 0) bulk_wait_group_read1();   // buffer's previous segment read
+                for (int pair = 0; pair < D / 64; ++pair) {
+                    uint32_t v[64];
+                    tmem_ld32(tl + C::kColdQ + 64 * pair, *reinterpret_cast<uint32_t(*)[32]>(v));
+                    tmem_ld32(tl + C::kColdQ + 64 * pair + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                    tmem_ld_wait();
+                    if (pair == D / 64 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(&bars->dq_free);
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int sg = 2 * pair + hh;                 // columns 32sg..32sg+31
+                        uint8_t* buf = stage + hh * 4096;
+                        if (sg >= 2) {
+                            if (lane == 0) bulk_wait_group_read1();   // buffer's previous segment read
+                            __syncwarp();
+                        }
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                                make_uint4(v[32 * hh + 4 * k], v[32 * hh + 4 * k + 1],
+                                           v[32 * hh + 4 * k + 2], v[32 * hh + 4 * k + 3]);
+                        fence_proxy_async_smem();
                         __syncwarp();
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                            make_uint4(v[32 * hh + 4 * k], v[32 * hh + 4 * k + 1],
-                                       v[32 * hh + 4 * k + 2], v[32 * hh + 4 * k + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_reduce_add_3d(&tmdQacc, buf, 32 * g, row0, bh);
-                        bulk_commit_group();
+                        if (lane == 0) {
+                            tma_reduce_add_3d(&tmdQacc, buf, 32 * sg, row0, it.bh);
+                            bulk_commit_group();
+                        }
                     }
                 }
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                mbar_arrive(&bars->ds_smem_free);
             }
-            if (lane == 0) bulk_wait_group_read0();
-            __syncwarp();
-            mbar_arrive(&bars->ds_smem_free);
         }
         // The CTA may exit once the TMA has read its shared-memory sources;
         // the reduce-adds themselves complete before the grid does.

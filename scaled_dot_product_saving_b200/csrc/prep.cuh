@@ -5,8 +5,9 @@
 //   O(n dv) instead of O(n m). It also writes the forward's LSE in base 2,
 //   and both arrays are padded to whole 128-row tiles (D = 0 and LSE = +inf
 //   in the padding, so padded query rows get P = 0 on the tensor-core path).
-//   The same launch zeroes the fp32 dQ accumulator. D is stored multiplied by
-//   `d_scale` (the tensor-core backward folds the attention scale into it).
+//   The same launch zeroes the fp32 dQ accumulator and the tensor-core
+//   backward's work-item counter. D is stored multiplied by `d_scale` (the
+//   tensor-core backward folds the attention scale into it).
 // finalize: dQ = post_scale * dQacc, converted to the element type.
 #pragma once
 
@@ -40,8 +41,9 @@ __device__ __forceinline__ float row_dot_bf16_vec(const __nv_bfloat16* o, const 
 __global__ void __launch_bounds__(kThreads)
 preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                     const float* __restrict__ LSE, float* __restrict__ lse2,
-                    float* __restrict__ Dd, float* __restrict__ dQacc, size_t dq_elems,
-                    int BH, int n, int n_pad, int dv, float d_scale) {
+                    float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ sched,
+                    size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
     const int G = dv / 8;                       // lanes per row
     const int rows_per_warp = 32 / G;
     const int lane = threadIdx.x & 31;
@@ -84,8 +86,9 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 preprocess_generic(const T* __restrict__ O, const T* __restrict__ dO,
                    const float* __restrict__ LSE, float* __restrict__ lse2,
-                   float* __restrict__ Dd, float* __restrict__ dQacc, size_t dq_elems, int BH,
-                   int n, int n_pad, int dv, float d_scale) {
+                   float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ sched,
+                   size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
     const int lane = threadIdx.x & 31;
     const size_t warp_global = (size_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const size_t nwarps = (size_t(gridDim.x) * kThreads) >> 5;
