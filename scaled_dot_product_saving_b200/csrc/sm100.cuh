@@ -105,6 +105,35 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
     return __all_sync(0xffffffffu, ok);
 }
 
+// ------------------------------------------------- cluster launch control
+// Ask the hardware to cancel the launch of a CTA of this grid that has not
+// started yet; the 16-byte answer is written to `resp` (16-byte aligned shared
+// memory) and signals `bar` with 16 transaction bytes. After an answer that
+// reports no cancellation, no further request may be made.
+__device__ __forceinline__ void clc_try_cancel(void* resp, uint64_t* bar) {
+    asm volatile(
+        "clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 "
+        "[%0], [%1];" ::"r"(smem_addr(resp)),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+// Decode an answer: true and the cancelled CTA's x index if a CTA was
+// cancelled (its work is now the caller's), false if none was left.
+__device__ __forceinline__ bool clc_query(const void* resp, int* ctaid_x) {
+    uint32_t ok, x;
+    asm volatile(
+        "{\n\t.reg .b128 r;\n\t.reg .pred p;\n\t"
+        "ld.shared.b128 r, [%2];\n\t"
+        "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t"
+        "clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, r;\n\t}"
+        : "=r"(ok), "=r"(x)
+        : "r"(smem_addr(resp))
+        : "memory");
+    *ctaid_x = int(x);
+    return ok != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 // Tiled 3-D load (coordinates innermost first) that signals `bar` with the
 // byte count when it lands. The innermost coordinate times the element size
