@@ -376,6 +376,39 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const uint32_t sK = smem_addr(smem + C::kOffK);
         const uint32_t sV = smem_addr(smem + C::kOffV);
         const uint32_t sdS = smem_addr(smem + C::kOffdS);
+        // dP^T(g) = V dO(g)^T once Q/dO(g) are in; its columns are free once
+        // the previous tile's dK MMAs (issued earlier) have read dS^T.
+        auto issue_dP = [&](int g) -> bool {
+            const int s = g % C::kStages;
+            if (!mbar_wait(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
+            tc_fence_after();
+            const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
+            }
+            return true;
+        };
+        // S^T(g) = K Q(g)^T (issued after dP^T(g)); s_full then reports both.
+        // At d = 128 its columns hold the previous tile's dQ until the dQ
+        // warpgroup has read it out.
+        auto issue_S = [&](int g) -> bool {
+            if (C::kAlias && g > 0 &&
+                !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns))
+                return false;
+            tc_fence_after();
+            const uint32_t sQ = smem_addr(smem + C::kOffQ + (g % C::kStages) * C::kTileBytes);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
+                       sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
+            }
+            mma_commit(&bars->s_full);
+            return true;
+        };
         bool ok = true;
         int g = 0;
         for (int j = 0; ok; ++j) {
@@ -387,37 +420,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 ok = false;
                 break;
             }
+            // At d = 64 (dQ in columns of its own) the next tile's dP^T and S^T
+            // are issued right after this tile's dV/dK MMAs, before the dQ MMA
+            // waits for the dS tile, so the P/dS warps start on tile t+1 while
+            // dS(t) reaches shared memory. At d = 128 the dQ MMA goes first:
+            // its result paces the dQ reduce-adds, whose staging holds the dS
+            // tile (issuing dP^T first measured 8 % slower).
+            bool ahead = false;
             for (int t = 0; t < T; ++t, ++g) {
                 const int s = g % C::kStages;
                 const uint32_t sQ = smem_addr(smem + C::kOffQ + s * C::kTileBytes);
                 const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
-                if (!mbar_wait(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                // dP^T first: its columns are free once the previous dK MMAs
-                // (issued earlier) have read dS^T from them.
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                           sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
-                }
-                // S^T shares its columns with the previous tile's dQ (d = 128).
-                if (C::kAlias && g > 0 &&
-                    !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                    mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
-                           sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
-                }
-                mma_commit(&bars->s_full);
+                if (!ahead && !issue_dP(g)) { ok = false; break; }
+                if (!ahead && !issue_S(g)) { ok = false; break; }
+                ahead = false;
                 // The item's first dV/dK MMAs overwrite the accumulators: the
                 // previous item's epilogue must have read them out.
                 if (t == 0 && j > 0 &&
@@ -449,6 +465,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 if (!ok) break;
                 mma_commit(&bars->q_empty[s]);
                 if (t == T - 1) mma_commit(&bars->acc_done);
+                if (!C::kAlias && t + 1 < T) {
+                    if (!issue_dP(g + 1) || !issue_S(g + 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ahead = true;
+                }
                 if (!C::kAlias && g > 0 &&
                     !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
