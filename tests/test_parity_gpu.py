@@ -69,6 +69,18 @@ def test_cuda_core_path_bf16(d, causal):
     _assert_within(full_compare(w), TOL["bf16"], w.name)
 
 
+@pytest.mark.parametrize("B,H,n,m,d,causal", [
+    (2, 40, 700, 700, 128, True),      # 240 forward / 480 backward items: several per CTA, ragged
+    (4, 50, 300, 1000, 64, False),     # 400 / 1600 items, n != m, both ragged
+    (1, 160, 130, 130, 128, True),     # one-key-tile items and one-tile pairs (has no tile B)
+])
+def test_persistent_many_items(B, H, n, m, d, causal):
+    """Problems with more work items than SMs, so that every persistent CTA
+    walks several items of different lengths (every head compared in full)."""
+    w = synth.make_small(B, H, n, m, d, d, "bf16", causal, seed=B * H + n + d)
+    _assert_within(full_compare(w), TOL["bf16"], w.name)
+
+
 @pytest.mark.parametrize("d,causal,scale", [
     (128, True, -0.09),    # negative scale: the softmax keeps the smallest raw score
     (64, False, -0.3),
