@@ -1,8 +1,9 @@
 // bwd_tc.cuh -- tensor-core backward for bf16, d == dv in {64, 128}.
 //
-// Key-tile major. One CTA owns 128 keys (K_j, V_j resident in shared memory)
-// of one (batch, head) and walks the 128-row query tiles i that can see them
-// (i >= j when causal). Per query tile, with keys as the MMA's M dimension:
+// Key-tile major. A work item is 128 keys (K_j, V_j resident in shared memory)
+// of one (batch, head) and the 128-row query tiles i that can see them (i >= j
+// when causal); persistent CTAs, one per SM, take the items in order from a
+// counter (see the kernel). Per query tile, with keys as the MMA's M dimension:
 //   S^T  = K_j Q_i^T                  tcgen05 (A = K_j, B = Q_i, both K-major)
 //   dP^T = V_j dO_i^T                 tcgen05 (A = V_j, B = dO_i)
 //   P^T  = 2^(S^T*scale*log2e - LSE_i*log2e), 0 where masked
@@ -27,9 +28,10 @@
 // columns, so no chunk overwrites data another chunk has yet to read. dS for
 // the dQ MMA is kept in registers and written to shared memory only at the
 // end of the tile, by when the dQ warpgroup has normally finished staging the
-// previous tile's dQ through that buffer. CTAs are ordered head-major, so the
+// previous tile's dQ through that buffer. Items are ordered head-major, so the
 // key tiles of one head run together and share its Q/dO tiles and its slice
-// of the dQ accumulator through L2.
+// of the dQ accumulator through L2. An item's dV/dK epilogue is staged in the
+// Q/dO stage of its last tile and overlaps the next item's first loads.
 //
 // Where the pages stand: dV, dP, dS, dQ and dK are "Attention Backward Pass
 // (dQ, dK, dV)", section "Backward", and "Attention backward", Problems 2-6;
@@ -44,11 +46,11 @@
 //
 // TMEM (512 columns). d = 128: dV [0,128) dK [128,256) S^T [256,384)
 // dP^T [384,512); chunk c's P^T (bf16) goes to [256+32c, 256+32c+16) and its
-// dS^T to [384+32c, 384+32c+16); dQ then takes all of [256,384). The tensor pipe runs MMAs in issue order, so the dQ
-// MMA, issued after the last dV MMA, overwrites P^T only once it has been
-// read; the next tile's dP^T MMA is issued before the dQ drain is awaited and
-// only its S^T MMA waits for it. d = 64: dV [0,64) dK [64,128) S^T [128,256)
-// dP^T [256,384) dQ [384,448).
+// dS^T to [384+32c, 384+32c+16); dQ then takes all of [256,384). The tensor
+// pipe runs MMAs in issue order, so the dQ MMA, issued after the last dV MMA,
+// overwrites P^T only once it has been read; the next tile's dP^T MMA is
+// issued before the dQ drain is awaited and only its S^T MMA waits for it.
+// d = 64: dV [0,64) dK [64,128) S^T [128,256) dP^T [256,384) dQ [384,448).
 #pragma once
 
 #include "sm100.cuh"
@@ -56,7 +58,7 @@
 namespace attn {
 namespace bwdtc {
 
-constexpr int kBN = 128;      // keys per CTA
+constexpr int kBN = 128;      // keys per work item
 constexpr int kBM = 128;      // queries per tile
 constexpr int kChunks = 4;    // 32-query chunks of a tile
 constexpr int kThreads = 448;

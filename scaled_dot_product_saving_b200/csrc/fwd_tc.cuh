@@ -5,11 +5,13 @@
 // Pass (dQ, dK, dV)", section on the forward; under the causal mask key j > i
 // is excluded before the softmax).
 //
-// One CTA computes two adjacent 128-row query tiles, A = 2p and B = 2p + 1,
-// of one (batch, head), sharing every key and value tile it loads; under the
-// causal mask B needs one key tile more than A. CTAs run in groups of heads
+// A work item is two adjacent 128-row query tiles, A = 2p and B = 2p + 1, of
+// one (batch, head), sharing every key and value tile loaded for it; under the
+// causal mask B needs one key tile more than A. Items run in groups of heads
 // (so a group's keys and values stay in L2), heaviest query rows first within
-// a group. For each 128-key tile t and each query tile x:
+// a group. The grid has one CTA per item, but the CTAs are persistent: each
+// takes over the items of CTAs not yet launched through cluster launch control
+// (see the kernel). For each 128-key tile t and each query tile x:
 //   S_x = Q_x K_t^T          tcgen05.mma, both operands K-major in shared
 //                            memory, fp32 accumulator in TMEM
 //   P_x = 2^(S_x * scale * log2e - m_x)   one softmax warpgroup per query
@@ -39,8 +41,9 @@
 // warp 9 TMEM allocator and MMA issuer.
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+d),
 // O_B [256+d, 256+2d).
-// Shared memory: Q_A, Q_B, then K and V rings with their own barriers (a K
-// tile is released as soon as both S products that read it are done).
+// Shared memory: Q_A, Q_B (each also the staging buffer of its O epilogue),
+// then K and V rings with their own barriers (a K tile is released as soon as
+// both S products that read it are done).
 #pragma once
 
 #include "sm100.cuh"
