@@ -38,6 +38,14 @@ therefore apply the definition to ``row_block`` query rows at a time, so that
 the n x m score matrix of a long sequence never has to exist at once.
 Within a block nothing is fused or reordered.
 
+Projection and input gradients of self-attention ("Lesson 4 - The Backward
+Pass for Attention", section "Step 4: Back to the Parameters and Input";
+"Attention backward", Problem 7), with Q = X Wq, K = X Wk, V = X Wv and the
+H heads taken as consecutive column blocks of each projection:
+      dWq = sum over the batch of X^T dQ   (likewise dWk, dWv)
+      dX  = dQ Wq^T + dK Wk^T + dV Wv^T    (X feeds all three projections)
+with dQ, dK, dV merged back from heads to columns.
+
 Pins (tests/test_oracle.py): the worked examples of "Attention Backward Pass
 (dQ, dK, dV)" (section "Examples"); the loss value printed in "Lesson 4 - The
 Backward Pass for Attention" (section "A Scalar Loss So dout Is Known"),
@@ -61,6 +69,8 @@ __all__ = [
     "grad_v", "grad_p", "softmax_jvp", "grad_q", "grad_k",
     "head_forward", "head_backward",
     "attention_forward", "attention_backward",
+    "split_heads", "merge_heads", "project_qkv", "grad_weight", "grad_input",
+    "projection_backward",
 ]
 
 ROW_BLOCK = 256
@@ -218,3 +228,48 @@ def attention_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOC
                                             scale, row_block)
     return (dQ.reshape(lead + dQ.shape[1:]), dK.reshape(lead + dK.shape[1:]),
             dV.reshape(lead + dV.shape[1:]))
+
+
+# --------------------------------------------------------------------------
+# Projection and input gradients ("Lesson 4", Step 4; "Attention backward",
+# Problem 7)
+# --------------------------------------------------------------------------
+def split_heads(T: np.ndarray, H: int) -> np.ndarray:
+    """[B, n, H*w] -> [B, H, n, w]: head h is column block h of a projection."""
+    B, n, HW = T.shape
+    return T.reshape(B, n, H, HW // H).transpose(0, 2, 1, 3)
+
+
+def merge_heads(T: np.ndarray) -> np.ndarray:
+    """[B, H, n, w] -> [B, n, H*w], the inverse of split_heads."""
+    B, H, n, w = T.shape
+    return T.transpose(0, 2, 1, 3).reshape(B, n, H * w)
+
+
+def project_qkv(X, Wq, Wk, Wv, H):
+    """Q, K, V = X Wq, X Wk, X Wv, split into H heads (Problem 7's forward)."""
+    X = np.asarray(X, dtype=np.float64)
+    return (split_heads(X @ Wq, H), split_heads(X @ Wk, H), split_heads(X @ Wv, H))
+
+
+def grad_weight(X: np.ndarray, dT: np.ndarray) -> np.ndarray:
+    """dW = sum over the batch of X_b^T dT_b for T = X W: the weight is shared
+    across the batch, so its gradient sums the per-item contributions
+    ("Lesson 4", Step 4). X [B, n, C], dT [B, n, w] -> [C, w]."""
+    return np.einsum("bnc,bnw->cw", X, dT)
+
+
+def grad_input(dQm, dKm, dVm, Wq, Wk, Wv) -> np.ndarray:
+    """dX = dQ Wq^T + dK Wk^T + dV Wv^T: X feeds all three projections and
+    the three paths add (Problem 7). Gradients merged to [B, n, H*w]."""
+    return dQm @ Wq.T + dKm @ Wk.T + dVm @ Wv.T
+
+
+def projection_backward(X, Wq, Wk, Wv, dQ, dK, dV):
+    """(dX, dWq, dWk, dWv) from dQ, dK, dV shaped [B, H, n, w] (the heads as
+    split by project_qkv)."""
+    X = np.asarray(X, dtype=np.float64)
+    Wq, Wk, Wv = (np.asarray(W, dtype=np.float64) for W in (Wq, Wk, Wv))
+    dQm, dKm, dVm = (merge_heads(np.asarray(G, dtype=np.float64)) for G in (dQ, dK, dV))
+    return (grad_input(dQm, dKm, dVm, Wq, Wk, Wv),
+            grad_weight(X, dQm), grad_weight(X, dKm), grad_weight(X, dVm))

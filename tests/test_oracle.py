@@ -102,13 +102,10 @@ def test_lesson4_gradient_check_through_projections():
     chain rule, written here in the test) pass the page's gradient check."""
     _, X, Wq, Wk, Wv, G = _lesson4_setup()
     spec = golden()["lesson4_gradient_check"]
-    dQ, dK, dV = ref.attention_backward(X @ Wq, X @ Wk, X @ Wv, G)
-    grads = {
-        "dWq": np.einsum("btc,bth->ch", X, dQ),
-        "dWk": np.einsum("btc,bth->ch", X, dK),
-        "dWv": np.einsum("btc,bth->ch", X, dV),
-        "dX": dQ @ Wq.T + dK @ Wk.T + dV @ Wv.T,
-    }
+    Q, K, V = ref.project_qkv(X, Wq, Wk, Wv, 1)
+    dQ, dK, dV = ref.attention_backward(Q, K, V, ref.split_heads(G, 1))
+    dX, dWq, dWk, dWv = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)
+    grads = {"dWq": dWq, "dWk": dWk, "dWv": dWv, "dX": dX}
     params = {"dWq": Wq, "dWk": Wk, "dWv": Wv, "dX": X}
     eps = spec["eps"]
     for name, p in params.items():
@@ -446,3 +443,94 @@ def test_unstable_softmax_is_caught(monkeypatch):
     with np.errstate(all="ignore"):
         bad, _ = ref.head_forward(Q, K, V, scale=1.0)
     assert not np.allclose(good, bad, equal_nan=False)
+
+
+# --------------------------------------------------------------------------
+# Projection gradients with several heads (Problem 7 per head; Problem 10's
+# column blocks)
+# --------------------------------------------------------------------------
+def _mh_setup(seed=7, B=2, n=5, C=6, H=3, d=2, dv=3):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((B, n, C))
+    Wq = rng.standard_normal((C, H * d)) * 0.5
+    Wk = rng.standard_normal((C, H * d)) * 0.5
+    Wv = rng.standard_normal((C, H * dv)) * 0.5
+    G = rng.standard_normal((B, n, H * dv))
+    return X, Wq, Wk, Wv, G
+
+
+def _mh_loss(X, Wq, Wk, Wv, G, causal, H=3):
+    Q, K, V = ref.project_qkv(X, Wq, Wk, Wv, H)
+    O, _ = ref.attention_forward(Q, K, V, causal)
+    return float(np.sum(ref.merge_heads(O) * G))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_projection_backward_multihead_finite_differences(causal):
+    """Every entry of dX, dWq, dWk, dWv of a three-head self-attention against
+    central differences of L = sum(merge(O) * G)."""
+    X, Wq, Wk, Wv, G = _mh_setup()
+    H = 3
+    Q, K, V = ref.project_qkv(X, Wq, Wk, Wv, H)
+    dQ, dK, dV = ref.attention_backward(Q, K, V, ref.split_heads(G, H), causal)
+    grads = dict(zip(("dX", "dWq", "dWk", "dWv"),
+                     ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)))
+    params = {"dX": X, "dWq": Wq, "dWk": Wk, "dWv": Wv}
+    eps = 1e-6
+    for name, p in params.items():
+        assert grads[name].shape == p.shape, name
+        num = np.zeros_like(p)
+        for idx in np.ndindex(p.shape):
+            orig = p[idx]
+            p[idx] = orig + eps
+            lp = _mh_loss(X, Wq, Wk, Wv, G, causal)
+            p[idx] = orig - eps
+            lm = _mh_loss(X, Wq, Wk, Wv, G, causal)
+            p[idx] = orig
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grads[name], num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_split_merge_heads_layout():
+    """Head h is column block h: split then merge is the identity, and head
+    h's rows are X Wq[:, h*d:(h+1)*d]."""
+    X, Wq, Wk, Wv, _ = _mh_setup()
+    Q, _, _ = ref.project_qkv(X, Wq, Wk, Wv, 3)
+    np.testing.assert_array_equal(ref.merge_heads(Q), X @ Wq)
+    np.testing.assert_allclose(Q[:, 1], X @ Wq[:, 2:4], rtol=0, atol=1e-14)
+
+
+def test_projection_backward_mutants_fail(monkeypatch):
+    """The pages' two projection mistakes, planted in the oracle, fail the
+    finite-difference pin: a path through X left out, and a transposed
+    weight gradient."""
+    X, Wq, Wk, Wv, G = _mh_setup(seed=11, C=4, H=2, d=2, dv=2)
+    H = 2
+    Q, K, V = ref.project_qkv(X, Wq, Wk, Wv, H)
+    dQ, dK, dV = ref.attention_backward(Q, K, V, ref.split_heads(G, H))
+    eps = 1e-6
+
+    def fd_dx():
+        num = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            orig = X[idx]
+            X[idx] = orig + eps
+            lp = float(np.sum(ref.merge_heads(ref.attention_forward(*ref.project_qkv(X, Wq, Wk, Wv, H))[0]) * G))
+            X[idx] = orig - eps
+            lm = float(np.sum(ref.merge_heads(ref.attention_forward(*ref.project_qkv(X, Wq, Wk, Wv, H))[0]) * G))
+            X[idx] = orig
+            num[idx] = (lp - lm) / (2 * eps)
+        return num
+
+    num = fd_dx()
+    good = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)[0]
+    np.testing.assert_allclose(good, num, rtol=1e-6, atol=1e-8)
+    monkeypatch.setattr(ref, "grad_input", lambda dQm, dKm, dVm, Wq, Wk, Wv: dQm @ Wq.T + dVm @ Wv.T)
+    bad = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)[0]
+    assert np.max(np.abs(bad - num)) > 1e-3
+    # C == H*d here, so the transposed product has the right shape
+    monkeypatch.setattr(ref, "grad_weight", lambda X, dT: np.einsum("bnc,bnw->wc", X, dT))
+    dWq_bad = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)[1]
+    monkeypatch.undo()
+    dWq_good = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)[1]
+    assert np.max(np.abs(dWq_bad - dWq_good)) > 1e-3
