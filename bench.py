@@ -53,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=16)
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--proj", action="store_true",
+                   help="time attn_proj_bwd (projection and input gradients) instead")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -383,6 +385,79 @@ def run_ours(args, w, rank, world, local):
 
 
 # ---------------------------------------------------------------- oracle timing
+PROJ_SHAPE = dict(B=2, n=4096, d_model=4096, H=32, d=128, dv=128)
+
+
+def run_proj(args, rank, world, local):
+    """attn_proj_bwd at the headline attention shape with d_model = H*d:
+    dX = [dQ|dK|dV] [Wq|Wk|Wv]^T and dWq, dWk, dWv = X^T dQ, ... over all
+    B*n tokens. Inputs are synthetic bf16 normals, resident in HBM."""
+    import scaled_dot_product_saving_b200 as lib
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c = PROJ_SHAPE
+    B, n, d_model, H, d, dv = c["B"], c["n"], c["d_model"], c["H"], c["d"], c["dv"]
+    g = torch.Generator().manual_seed(7 + 1000 * rank)
+
+    def r(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g) * std).to(torch.bfloat16).to(dev)
+    X = r(B, n, d_model)
+    Wq, Wk, Wv = (r(d_model, H * w_, std=d_model ** -0.5) for w_ in (d, d, dv))
+    dQ, dK, dV = r(B, H, n, d), r(B, H, n, d), r(B, H, n, dv)
+    outs = [torch.empty_like(t) for t in (X, Wq, Wk, Wv)]
+    ws = torch.empty(lib.attn_proj_bwd_workspace_size(B, n, d_model, H, d, dv, 1),
+                     dtype=torch.uint8, device=dev)
+    tokens, wtot = B * n, 2 * H * d + H * dv
+    flops = 2.0 * tokens * d_model * wtot * 2      # dX and the three dW, same count each
+
+    def step():
+        lib.attn_proj_bwd(X, Wq, Wk, Wv, dQ, dK, dV, workspace=ws, dx=outs[0], dwq=outs[1],
+                          dwk=outs[2], dwv=outs[3])
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    sampler.start()
+    lib.attn_trace_begin(min(65536, 16 * args.steps))
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world, local)
+    sampler.stop()
+    trace = lib.attn_trace_end()
+    if lib.attn_get_device_error() != 0:
+        raise RuntimeError("device-side timeout in the timed region")
+    (slow_ms,) = max_over_ranks([t0.elapsed_time(t1)], world, dev)
+    gemm_ms = sum(ms for name, ms in trace if name == "gemm") / args.steps
+    gather_ms = sum(ms for name, ms in trace if name == "proj_gather") / args.steps
+    peaks, peaks_src = measured_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    if rank != 0:
+        return None
+    return {
+        "metric": "attention projection-gradient TFLOP/s (bf16)",
+        "value": world * args.steps * flops / (slow_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(slow_ms / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "proj_b2n4096_dmodel4096_h32_d128", **c,
+                   "parallelism": "replicas" if world > 1 else "none"},
+        "kernel_ms": {"gemm": round(gemm_ms, 4), "proj_gather": round(gather_ms, 4)},
+        "roofline": {"bound": "tensor", "kernel": "gemm (4 launches a step)",
+                     "achieved": round(achieved, 3), "peak": peak,
+                     "peak_source": f"bf16_tflops ({peaks_src}, burst)", "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": None},
+        "gpu_launches": sum(1 for _ in trace),
+        "clocks": sampler.summary(),
+    }
+
+
 def oracle_sample(w, seconds, max_heads=None):
     """Time the oracle backward on whole heads of the workload until `seconds`
     have passed. Returns (TFLOP/s in the metric's counting, heads, elapsed)."""
@@ -444,7 +519,9 @@ def main(argv=None):
     w = synth.workload(args.workload)
     rank, world, local = init_distributed()
     try:
-        if args.impl == "reference":
+        if args.proj:
+            out = run_proj(args, rank, world, local)
+        elif args.impl == "reference":
             out = run_reference(args, w, rank, world)
         else:
             out = run_ours(args, w, rank, world, local)

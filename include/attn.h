@@ -177,7 +177,9 @@ typedef enum {
     ATTN_KERNEL_PREPROCESS = 3,   /* D = rowsum(dO*O), base-2 LSE, zero dQacc */
     ATTN_KERNEL_BWD_TENSOR = 4,   /* tcgen05 backward                         */
     ATTN_KERNEL_BWD_SIMT = 5,     /* CUDA-core backward                       */
-    ATTN_KERNEL_FINALIZE = 6      /* dQ accumulator -> dQ                      */
+    ATTN_KERNEL_FINALIZE = 6,     /* dQ accumulator -> dQ                      */
+    ATTN_KERNEL_PROJ_GATHER = 7,  /* per-head gradients / weights side by side */
+    ATTN_KERNEL_GEMM = 8          /* tcgen05 GEMM of the projection gradients  */
 } attn_kernel_id_t;
 
 typedef struct {
@@ -188,10 +190,41 @@ typedef struct {
 attn_status_t attn_trace_begin(int capacity);
 int attn_trace_end(attn_kernel_time_t* out, int max_entries);
 
+/*
+ * Projection and input gradients of multi-head self-attention ("Lesson 4 -
+ * The Backward Pass for Attention", section "Step 4: Back to the Parameters
+ * and Input"; "Attention backward", Problem 7). With Q = X Wq, K = X Wk,
+ * V = X Wv and head h the column block h of each projection (Q [B,n,H*d]
+ * split into [B,H,n,d], as attn_fwd/attn_bwd take it), and dQ, dK, dV from
+ * attn_bwd:
+ *   dWq = sum over the batch of X_b^T dQ_b   [d_model, H*d]   (same for dWk;
+ *   dWv [d_model, H*dv])
+ *   dX  = dQ Wq^T + dK Wk^T + dV Wv^T        [B, n, d_model]
+ * with dQ, dK, dV merged back to [B, n, H*w]. Arguments:
+ *   X [B,n,d_model], Wq, Wk [d_model, H*d], Wv [d_model, H*dv]  (read only)
+ *   dQ, dK [B,H,n,d], dV [B,H,n,dv]                              (read only)
+ *   dX, dWq, dWk, dWv: outputs with the shapes of X, Wq, Wk, Wv  (written)
+ *   bf16 only (ATTN_ERR_UNSUPPORTED otherwise); fp32 accumulation; d, dv and
+ *   d_model multiples of 8 (ATTN_ERR_SHAPE otherwise); all pointers 16-byte
+ *   aligned; contiguous row-major tensors.
+ *   workspace: caller-owned device memory of attn_proj_bwd_workspace_size()
+ *   bytes (token-major copies of the gradients and the weights side by side);
+ *   contents on entry do not matter. Stream-ordered and asynchronous; a
+ *   non-OK status means nothing was launched.
+ */
+size_t attn_proj_bwd_workspace_size(int B, int n, int d_model, int H, int d, int dv,
+                                    attn_dtype_t dtype);
+attn_status_t attn_proj_bwd(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                            const void* dQ, const void* dK, const void* dV, void* dX,
+                            void* dWq, void* dWk, void* dWv, void* workspace,
+                            size_t workspace_bytes, int B, int n, int d_model, int H, int d,
+                            int dv, attn_dtype_t dtype, void* stream);
+
 /* Select the kernel path for later calls (see attn_path_t). */
 attn_status_t attn_set_path(attn_path_t path);
 
-/* Number of kernels the last successful attn_fwd/attn_bwd call launched. */
+/* Number of kernels the last successful attn_fwd/attn_bwd/attn_proj_bwd call
+ * launched. */
 int attn_last_launch_count(void);
 
 /* A static, human-readable name for a status code. */

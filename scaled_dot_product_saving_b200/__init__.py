@@ -23,6 +23,7 @@ __all__ = [
     "attn_probe_timeout", "attn_set_path", "attn_last_launch_count", "attn_status_string",
     "dtype_code", "attn_trace_begin", "attn_trace_end", "KERNEL_NAMES",
     "attn_bwd_noalloc", "attn_bwd_noalloc_scratch_bytes",
+    "attn_proj_bwd", "attn_proj_bwd_workspace_size",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
@@ -33,7 +34,7 @@ ATTN_OK = 0
 ATTN_ERR_DEVICE_TIMEOUT = 8
 
 KERNEL_NAMES = {1: "fwd_tensor", 2: "fwd_simt", 3: "preprocess", 4: "bwd_tensor",
-                5: "bwd_simt", 6: "finalize"}
+                5: "bwd_simt", 6: "finalize", 7: "proj_gather", 8: "gemm"}
 
 
 class _KernelTime(ctypes.Structure):
@@ -87,6 +88,11 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.attn_bwd_noalloc.restype = i
     L.attn_bwd_noalloc_scratch_bytes.argtypes = []
     L.attn_bwd_noalloc_scratch_bytes.restype = sz
+    L.attn_proj_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
+    L.attn_proj_bwd_workspace_size.restype = sz
+    L.attn_proj_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                i, i, i, i, i, i, i, vp]
+    L.attn_proj_bwd.restype = i
     return L
 
 
@@ -233,3 +239,37 @@ def attn_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, causal=False, scale=None, 
                                 _stream_handle(stream)),
            "attn_bwd_noalloc")
     return dq, dk, dv
+
+
+def attn_proj_bwd_workspace_size(B: int, n: int, d_model: int, H: int, d: int, dv: int,
+                                 dtype_code_: int) -> int:
+    return int(lib.attn_proj_bwd_workspace_size(B, n, d_model, H, d, dv, dtype_code_))
+
+
+def attn_proj_bwd(x, wq, wk, wv, dq, dk, dv, workspace=None, dx=None, dwq=None, dwk=None,
+                  dwv=None, stream=None):
+    """Returns (dX, dWq, dWk, dWv) for X [B,n,d_model], Wq/Wk [d_model,H*d],
+    Wv [d_model,H*dv] and dQ/dK [B,H,n,d], dV [B,H,n,dv] (head h = column
+    block h of each projection)."""
+    _require(x, wq, wk, wv, dq, dk, dv)
+    B, n, d_model = x.shape
+    _, H, n2, d = dq.shape
+    dvw = dv.shape[-1]
+    if (n2 != n or tuple(dk.shape) != (B, H, n, d) or tuple(dv.shape) != (B, H, n, dvw)
+            or tuple(wq.shape) != (d_model, H * d) or tuple(wk.shape) != (d_model, H * d)
+            or tuple(wv.shape) != (d_model, H * dvw)):
+        raise ValueError("attn_proj_bwd: inconsistent shapes")
+    code = dtype_code(x.dtype)
+    need = attn_proj_bwd_workspace_size(B, n, d_model, H, d, dvw, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+    dx = torch.empty_like(x) if dx is None else dx
+    dwq = torch.empty_like(wq) if dwq is None else dwq
+    dwk = torch.empty_like(wk) if dwk is None else dwk
+    dwv = torch.empty_like(wv) if dwv is None else dwv
+    _check(lib.attn_proj_bwd(_ptr(x), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(dx), _ptr(dwq), _ptr(dwk), _ptr(dwv), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(),
+                             B, n, d_model, H, d, dvw, code, _stream_handle(stream)),
+           "attn_proj_bwd")
+    return dx, dwq, dwk, dwv

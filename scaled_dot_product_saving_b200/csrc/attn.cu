@@ -18,6 +18,8 @@
 #include "prep.cuh"
 #include "fwd_tc.cuh"
 #include "bwd_tc.cuh"
+#include "gemm_tc.cuh"
+#include "proj.cuh"
 
 namespace {
 
@@ -112,6 +114,22 @@ bool make_map_typed(CUtensorMap* map, const void* base, int width, int rows, int
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A bf16 matrix of `rows` x `width` whose rows are `row_stride` elements apart,
+// viewed as [1, rows, width] with the 128-byte swizzle and box_x x box_y boxes.
+bool make_map_rows(CUtensorMap* map, const void* base, int width, int rows, size_t row_stride,
+                   int box_x, int box_y) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(width), static_cast<cuuint64_t>(rows), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride) * 2,
+                             static_cast<cuuint64_t>(row_stride) * 2 * rows};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(box_y), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool make_map(CUtensorMap* map, const void* base, int width, int rows, int bh) {
@@ -330,6 +348,49 @@ __global__ void probe_timeout_kernel(unsigned long long budget_ns) {
 
 }  // namespace
 
+// ------------------------------------------------------ projection grads
+struct ProjWorkspace {
+    size_t acat_off, wcat_off, total;
+    int wtot;
+};
+
+ProjWorkspace carve_proj(int B, int n, int d_model, int H, int d, int dv) {
+    ProjWorkspace w;
+    w.wtot = 2 * H * d + H * dv;
+    w.acat_off = 0;
+    w.wcat_off = round_up(static_cast<size_t>(B) * n * w.wtot * 2, 256);
+    w.total = w.wcat_off + round_up(static_cast<size_t>(d_model) * w.wtot * 2, 256);
+    return w;
+}
+
+attn_status_t check_proj(int B, int n, int d_model, int H, int d, int dv, attn_dtype_t dtype) {
+    if (dtype != ATTN_F32 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+    if (B < 1 || n < 1 || d_model < 1 || H < 1 || d < 1 || dv < 1) return ATTN_ERR_SHAPE;
+    if (static_cast<long long>(B) * n >= (1ll << 31) || d_model >= (1 << 24) ||
+        static_cast<long long>(H) * (2 * d + dv) >= (1 << 24))
+        return ATTN_ERR_SHAPE;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (d % 8 || dv % 8 || d_model % 8) return ATTN_ERR_SHAPE;
+    return ATTN_OK;
+}
+
+template <bool AK, bool BK>
+attn_status_t gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* D, int M, int N, int K,
+                   int ldd, cudaStream_t st) {
+    auto kern = attn::gemmtc::gemm_kernel<AK, BK>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn::gemmtc::kSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    dim3 grid((M + attn::gemmtc::kBM - 1) / attn::gemmtc::kBM,
+              (N + attn::gemmtc::kBN - 1) / attn::gemmtc::kBN);
+    if (grid.y > 65535) return ATTN_ERR_SHAPE;
+    return traced(ATTN_KERNEL_GEMM, st, [&] {
+        kern<<<grid, attn::gemmtc::kThreads, attn::gemmtc::kSmemBytes, st>>>(
+            ma, mb, static_cast<__nv_bfloat16*>(D), M, N, K, ldd, kWaitBudgetNs);
+        return launched();
+    });
+}
+
 extern "C" {
 
 attn_status_t attn_set_path(attn_path_t path) {
@@ -469,6 +530,83 @@ attn_status_t attn_probe_timeout(unsigned timeout_us, void* stream) {
     if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_SHAPE;
     probe_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(1000ull * timeout_us);
     return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_proj_bwd_workspace_size(int B, int n, int d_model, int H, int d, int dv,
+                                    attn_dtype_t dtype) {
+    if (check_proj(B, n, d_model, H, d, dv, dtype) != ATTN_OK) return 0;
+    return carve_proj(B, n, d_model, H, d, dv).total;
+}
+
+attn_status_t attn_proj_bwd(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                            const void* dQ, const void* dK, const void* dV, void* dX,
+                            void* dWq, void* dWk, void* dWv, void* workspace,
+                            size_t workspace_bytes, int B, int n, int d_model, int H, int d,
+                            int dv, attn_dtype_t dtype, void* stream) {
+    attn_status_t s = check_proj(B, n, d_model, H, d, dv, dtype);
+    if (s != ATTN_OK) return s;
+    const void* ins[7] = {X, Wq, Wk, Wv, dQ, dK, dV};
+    void* outs[4] = {dX, dWq, dWk, dWv};
+    for (const void* p : ins)
+        if (!p) return ATTN_ERR_NULL;
+    for (void* p : outs)
+        if (!p) return ATTN_ERR_NULL;
+    for (const void* p : ins)
+        if (!aligned16(p)) return ATTN_ERR_ALIGN;
+    for (void* p : outs)
+        if (!aligned16(p)) return ATTN_ERR_ALIGN;
+    const ProjWorkspace w = carve_proj(B, n, d_model, H, d, dv);
+    if (!workspace || workspace_bytes < w.total) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+
+    cudaStream_t st = as_stream(stream);
+    auto* acat = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w.acat_off);
+    auto* wcat = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + w.wcat_off);
+    const int tokens = B * n;
+    const int hd = H * d, hdv = H * dv;
+
+    // Tensor maps first: nothing is launched unless all of them encode.
+    // dX = A [Wq|Wk|Wv]^T: A K-major [tokens][wtot], B K-major [d_model][wtot].
+    // dW = X^T A_block: A = X MN-major [tokens][d_model], B = the column block
+    // of A MN-major [tokens][width], rows wtot apart.
+    CUtensorMap m_acat, m_wcat, m_x, m_bq, m_bk, m_bv;
+    if (!make_map_rows(&m_acat, acat, w.wtot, tokens, w.wtot, 64, attn::gemmtc::kBM) ||
+        !make_map_rows(&m_wcat, wcat, w.wtot, d_model, w.wtot, 64, attn::gemmtc::kBN) ||
+        !make_map_rows(&m_x, X, d_model, tokens, d_model, 64, 64) ||
+        !make_map_rows(&m_bq, acat, hd, tokens, w.wtot, 64, 64) ||
+        !make_map_rows(&m_bk, acat + hd, hd, tokens, w.wtot, 64, 64) ||
+        !make_map_rows(&m_bv, acat + 2 * hd, hdv, tokens, w.wtot, 64, 64))
+        return ATTN_ERR_CUDA;
+
+    auto gather = [&](auto kernel_launch) {
+        return traced(ATTN_KERNEL_PROJ_GATHER, st, [&] {
+            kernel_launch();
+            return launched();
+        });
+    };
+    const int grid_g = 148 * 8;
+    const struct { const void* g; int w; int col0; } heads[3] = {{dQ, d, 0}, {dK, d, hd}, {dV, dv, 2 * hd}};
+    for (const auto& hh : heads) {
+        s = gather([&] {
+            attn::proj::heads_to_tokens<<<grid_g, attn::proj::kThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(hh.g), acat, B, H, n, hh.w, w.wtot, hh.col0);
+        });
+        if (s != ATTN_OK) return s;
+    }
+    const struct { const void* W; int cols; int col0; } ws3[3] = {{Wq, hd, 0}, {Wk, hd, hd}, {Wv, hdv, 2 * hd}};
+    for (const auto& ww : ws3) {
+        s = gather([&] {
+            attn::proj::concat_cols<<<grid_g, attn::proj::kThreads, 0, st>>>(
+                static_cast<const __nv_bfloat16*>(ww.W), wcat, d_model, ww.cols, w.wtot, ww.col0);
+        });
+        if (s != ATTN_OK) return s;
+    }
+    s = gemm<true, true>(m_acat, m_wcat, dX, tokens, d_model, w.wtot, d_model, st);
+    if (s == ATTN_OK) s = gemm<false, false>(m_x, m_bq, dWq, d_model, hd, tokens, hd, st);
+    if (s == ATTN_OK) s = gemm<false, false>(m_x, m_bk, dWk, d_model, hd, tokens, hd, st);
+    if (s == ATTN_OK) s = gemm<false, false>(m_x, m_bv, dWv, d_model, hdv, tokens, hdv, st);
+    if (s == ATTN_OK) g_last_launches = 10;
+    return s;
 }
 
 const char* attn_status_string(attn_status_t s) {

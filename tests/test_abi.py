@@ -118,3 +118,31 @@ def test_status_strings(L):
 def test_valid_call_without_a_device_reports_cuda_error(L):
     assert fwd(L) == 7
     assert fwd(L, dt=0) == 7
+
+
+def proj(L, x=P, dq=P, ws=P, wsb=1 << 40, B=2, n=64, d_model=64, H=2, d=64, dv=64, dt=1):
+    return L.lib.attn_proj_bwd(x, P, P, P, dq, P, P, P, P, P, P, ws, wsb, B, n, d_model, H, d,
+                               dv, dt, NUL)
+
+
+def test_argument_checks_projection(L):
+    assert proj(L, x=NUL) == 1                     # ATTN_ERR_NULL
+    assert proj(L, B=0) == 2                       # ATTN_ERR_SHAPE
+    assert proj(L, d=12) == 2                      # widths must be multiples of 8
+    assert proj(L, d_model=100) == 2
+    assert proj(L, dt=0) == 4                      # fp32: ATTN_ERR_UNSUPPORTED
+    assert proj(L, dt=7) == 3                      # ATTN_ERR_DTYPE
+    assert proj(L, dq=MIS) == 5                    # ATTN_ERR_ALIGN
+    assert proj(L, wsb=16) == 6                    # ATTN_ERR_WORKSPACE
+    assert proj(L, ws=NUL) == 6
+
+
+def test_projection_workspace_formula(L):
+    def expect(B, n, d_model, H, d, dv):
+        wtot = 2 * H * d + H * dv
+        r = lambda x: -(-x // 256) * 256
+        return r(B * n * wtot * 2) + r(d_model * wtot * 2)
+    for args in [(2, 64, 64, 2, 64, 64), (2, 4096, 4096, 32, 128, 128), (3, 77, 200, 3, 64, 40)]:
+        assert L.attn_proj_bwd_workspace_size(*args, 1) == expect(*args)
+    assert L.attn_proj_bwd_workspace_size(2, 64, 64, 2, 64, 64, 0) == 0
+    assert L.attn_proj_bwd_workspace_size(2, 64, 60, 2, 64, 64, 1) == 0
