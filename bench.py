@@ -438,6 +438,44 @@ def run_proj(args, rank, world, local):
     peaks, peaks_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (gemm_ms * 1e-3) / 1e12
+
+    # The output projection of Problem 10 at the same shape: dWo = O_cat^T G,
+    # dO = G Wo^T sliced into heads.
+    O = r(B, H, n, dv)
+    Wo = r(H * dv, d_model, std=(H * dv) ** -0.5)
+    Gy = r(B, n, d_model)
+    o_outs = [torch.empty_like(O), torch.empty_like(Wo)]
+    o_ws = torch.empty(lib.attn_outproj_bwd_workspace_size(B, n, d_model, H, dv, 1),
+                       dtype=torch.uint8, device=dev)
+    o_flops = 2.0 * tokens * d_model * (H * dv) * 2
+
+    def o_step():
+        lib.attn_outproj_bwd(O, Wo, Gy, workspace=o_ws, do=o_outs[0], dwo=o_outs[1])
+    for _ in range(args.warmup):
+        o_step()
+    torch.cuda.synchronize()
+    t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lib.attn_trace_begin(min(65536, 8 * args.steps))
+    t2.record()
+    for _ in range(args.steps):
+        o_step()
+    t3.record()
+    torch.cuda.synchronize()
+    o_trace = lib.attn_trace_end()
+    if lib.attn_get_device_error() != 0:
+        raise RuntimeError("device-side timeout in the output-projection timing")
+    (o_ms,) = max_over_ranks([t2.elapsed_time(t3)], world, dev)
+    o_gemm_ms = sum(ms for name, ms in o_trace if name == "gemm") / args.steps
+    outproj = {
+        "value": round(world * args.steps * o_flops / (o_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        "ms_per_step": round(o_ms / args.steps, 4),
+        "kernel_ms": {"gemm": round(o_gemm_ms, 4),
+                      "proj_gather": round(sum(ms for nm, ms in o_trace if nm == "proj_gather")
+                                           / args.steps, 4)},
+        "roofline": {"bound": "tensor", "achieved": round(o_flops / (o_gemm_ms * 1e-3) / 1e12, 3),
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(o_flops / (o_gemm_ms * 1e-3) / 1e12 / peak, 4)},
+    }
     if rank != 0:
         return None
     return {
@@ -455,6 +493,7 @@ def run_proj(args, rank, world, local):
                      "frac": round(achieved / peak, 4), "traffic": None},
         "gpu_launches": sum(1 for _ in trace),
         "clocks": sampler.summary(),
+        "outproj": outproj,
     }
 
 

@@ -220,11 +220,32 @@ attn_status_t attn_proj_bwd(const void* X, const void* Wq, const void* Wk, const
                             size_t workspace_bytes, int B, int n, int d_model, int H, int d,
                             int dv, attn_dtype_t dtype, void* stream);
 
+/*
+ * Gradients of the multi-head output projection ("Attention backward",
+ * Problem 10): with Y = [O_1 ... O_H] Wo (O_h the heads of attn_fwd's output,
+ * concatenated along columns) and G = dL/dY,
+ *   dWo  = [O_1 ... O_H]^T G          summed over the batch   [H*dv, d_model]
+ *   dO_h = columns h*dv .. (h+1)*dv of G Wo^T                  [B,H,n,dv]
+ * dO is what attn_bwd takes as its dO. Arguments:
+ *   O [B,H,n,dv], Wo [H*dv, d_model], G [B,n,d_model]  (read only)
+ *   dO [B,H,n,dv], dWo [H*dv, d_model]                  (written)
+ *   bf16 only (ATTN_ERR_UNSUPPORTED otherwise); dv and d_model multiples of 8
+ *   (ATTN_ERR_SHAPE otherwise); pointers 16-byte aligned; workspace of
+ *   attn_outproj_bwd_workspace_size() bytes (the merged O and G Wo^T), its
+ *   contents on entry irrelevant. Stream-ordered; a non-OK status means
+ *   nothing was launched.
+ */
+size_t attn_outproj_bwd_workspace_size(int B, int n, int d_model, int H, int dv,
+                                       attn_dtype_t dtype);
+attn_status_t attn_outproj_bwd(const void* O, const void* Wo, const void* G, void* dO, void* dWo,
+                               void* workspace, size_t workspace_bytes, int B, int n,
+                               int d_model, int H, int dv, attn_dtype_t dtype, void* stream);
+
 /* Select the kernel path for later calls (see attn_path_t). */
 attn_status_t attn_set_path(attn_path_t path);
 
-/* Number of kernels the last successful attn_fwd/attn_bwd/attn_proj_bwd call
- * launched. */
+/* Number of kernels the last successful attn_fwd/attn_bwd/attn_proj_bwd/
+ * attn_outproj_bwd call launched. */
 int attn_last_launch_count(void);
 
 /* A static, human-readable name for a status code. */

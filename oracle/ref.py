@@ -44,7 +44,10 @@ Pass for Attention", section "Step 4: Back to the Parameters and Input";
 H heads taken as consecutive column blocks of each projection:
       dWq = sum over the batch of X^T dQ   (likewise dWk, dWv)
       dX  = dQ Wq^T + dK Wk^T + dV Wv^T    (X feeds all three projections)
-with dQ, dK, dV merged back from heads to columns.
+with dQ, dK, dV merged back from heads to columns. The multi-head output
+projection ("Attention backward", Problem 10), Y = [O_1 ... O_H] Wo:
+      dWo  = [O_1 ... O_H]^T G
+      dO_h = columns h*dv .. (h+1)*dv of G Wo^T
 
 Pins (tests/test_oracle.py): the worked examples of "Attention Backward Pass
 (dQ, dK, dV)" (section "Examples"); the loss value printed in "Lesson 4 - The
@@ -70,7 +73,7 @@ __all__ = [
     "head_forward", "head_backward",
     "attention_forward", "attention_backward",
     "split_heads", "merge_heads", "project_qkv", "grad_weight", "grad_input",
-    "projection_backward",
+    "projection_backward", "output_projection", "output_projection_backward",
 ]
 
 ROW_BLOCK = 256
@@ -273,3 +276,21 @@ def projection_backward(X, Wq, Wk, Wv, dQ, dK, dV):
     dQm, dKm, dVm = (merge_heads(np.asarray(G, dtype=np.float64)) for G in (dQ, dK, dV))
     return (grad_input(dQm, dKm, dVm, Wq, Wk, Wv),
             grad_weight(X, dQm), grad_weight(X, dKm), grad_weight(X, dVm))
+
+
+def output_projection(O, Wo):
+    """Y = [O_1 ... O_H] Wo for O [B, H, n, dv], Wo [H*dv, d_model] (Problem 10)."""
+    return merge_heads(np.asarray(O, dtype=np.float64)) @ np.asarray(Wo, dtype=np.float64)
+
+
+def output_projection_backward(O, Wo, G):
+    """(dO, dWo) for Y = [O_1 ... O_H] Wo and G = dL/dY [B, n, d_model]:
+    dWo = [O_1 ... O_H]^T G summed over the batch, and dO_h the column block h
+    of G Wo^T, since the concatenation only copies entries (Problem 10)."""
+    O = np.asarray(O, dtype=np.float64)
+    Wo = np.asarray(Wo, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    H = O.shape[1]
+    dWo = grad_weight(merge_heads(O), G)
+    dO = split_heads(G @ Wo.T, H)
+    return dO, dWo

@@ -24,6 +24,7 @@ __all__ = [
     "dtype_code", "attn_trace_begin", "attn_trace_end", "KERNEL_NAMES",
     "attn_bwd_noalloc", "attn_bwd_noalloc_scratch_bytes",
     "attn_proj_bwd", "attn_proj_bwd_workspace_size",
+    "attn_outproj_bwd", "attn_outproj_bwd_workspace_size",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
@@ -93,6 +94,10 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.attn_proj_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                 i, i, i, i, i, i, i, vp]
     L.attn_proj_bwd.restype = i
+    L.attn_outproj_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.attn_outproj_bwd_workspace_size.restype = sz
+    L.attn_outproj_bwd.argtypes = [vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, i, vp]
+    L.attn_outproj_bwd.restype = i
     return L
 
 
@@ -273,3 +278,29 @@ def attn_proj_bwd(x, wq, wk, wv, dq, dk, dv, workspace=None, dx=None, dwq=None, 
                              B, n, d_model, H, d, dvw, code, _stream_handle(stream)),
            "attn_proj_bwd")
     return dx, dwq, dwk, dwv
+
+
+def attn_outproj_bwd_workspace_size(B: int, n: int, d_model: int, H: int, dv: int,
+                                    dtype_code_: int) -> int:
+    return int(lib.attn_outproj_bwd_workspace_size(B, n, d_model, H, dv, dtype_code_))
+
+
+def attn_outproj_bwd(o, wo, g, workspace=None, do=None, dwo=None, stream=None):
+    """Returns (dO, dWo) for Y = [O_1 ... O_H] Wo: O [B,H,n,dv], Wo [H*dv,d_model],
+    G = dL/dY [B,n,d_model]."""
+    _require(o, wo, g)
+    B, H, n, dvw = o.shape
+    d_model = g.shape[-1]
+    if tuple(g.shape) != (B, n, d_model) or tuple(wo.shape) != (H * dvw, d_model):
+        raise ValueError("attn_outproj_bwd: inconsistent shapes")
+    code = dtype_code(o.dtype)
+    need = attn_outproj_bwd_workspace_size(B, n, d_model, H, dvw, code)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=o.device)
+    do = torch.empty_like(o) if do is None else do
+    dwo = torch.empty_like(wo) if dwo is None else dwo
+    _check(lib.attn_outproj_bwd(_ptr(o), _ptr(wo), _ptr(g), _ptr(do), _ptr(dwo), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(),
+                                B, n, d_model, H, dvw, code, _stream_handle(stream)),
+           "attn_outproj_bwd")
+    return do, dwo

@@ -609,6 +609,55 @@ attn_status_t attn_proj_bwd(const void* X, const void* Wq, const void* Wk, const
     return s;
 }
 
+size_t attn_outproj_bwd_workspace_size(int B, int n, int d_model, int H, int dv,
+                                       attn_dtype_t dtype) {
+    if (check_proj(B, n, d_model, H, 8, dv, dtype) != ATTN_OK) return 0;
+    return 2 * round_up(static_cast<size_t>(B) * n * H * dv * 2, 256);
+}
+
+attn_status_t attn_outproj_bwd(const void* O, const void* Wo, const void* G, void* dO, void* dWo,
+                               void* workspace, size_t workspace_bytes, int B, int n,
+                               int d_model, int H, int dv, attn_dtype_t dtype, void* stream) {
+    attn_status_t s = check_proj(B, n, d_model, H, 8, dv, dtype);
+    if (s != ATTN_OK) return s;
+    if (!O || !Wo || !G || !dO || !dWo) return ATTN_ERR_NULL;
+    if (!aligned16(O) || !aligned16(Wo) || !aligned16(G) || !aligned16(dO) || !aligned16(dWo))
+        return ATTN_ERR_ALIGN;
+    const size_t half = round_up(static_cast<size_t>(B) * n * H * dv * 2, 256);
+    if (!workspace || workspace_bytes < 2 * half) return ATTN_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
+
+    cudaStream_t st = as_stream(stream);
+    auto* ocat = static_cast<__nv_bfloat16*>(workspace);
+    auto* docat = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + half);
+    const int tokens = B * n, hdv = H * dv;
+    // dWo = Ocat^T G: A = Ocat MN-major [tokens][hdv], B = G MN-major
+    // [tokens][d_model]. dOcat = G Wo^T: A = G K-major, B = Wo K-major
+    // [hdv][d_model].
+    CUtensorMap m_ocat, m_g_mn, m_g_k, m_wo;
+    if (!make_map_rows(&m_ocat, ocat, hdv, tokens, hdv, 64, 64) ||
+        !make_map_rows(&m_g_mn, G, d_model, tokens, d_model, 64, 64) ||
+        !make_map_rows(&m_g_k, G, d_model, tokens, d_model, 64, attn::gemmtc::kBM) ||
+        !make_map_rows(&m_wo, Wo, d_model, hdv, d_model, 64, attn::gemmtc::kBN))
+        return ATTN_ERR_CUDA;
+    const int grid_g = 148 * 8;
+    s = traced(ATTN_KERNEL_PROJ_GATHER, st, [&] {
+        attn::proj::heads_to_tokens<<<grid_g, attn::proj::kThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(O), ocat, B, H, n, dv, hdv, 0);
+        return launched();
+    });
+    if (s == ATTN_OK) s = gemm<false, false>(m_ocat, m_g_mn, dWo, hdv, d_model, tokens, d_model, st);
+    if (s == ATTN_OK) s = gemm<true, true>(m_g_k, m_wo, docat, tokens, hdv, d_model, hdv, st);
+    if (s == ATTN_OK)
+        s = traced(ATTN_KERNEL_PROJ_GATHER, st, [&] {
+            attn::proj::tokens_to_heads<<<grid_g, attn::proj::kThreads, 0, st>>>(
+                docat, static_cast<__nv_bfloat16*>(dO), B, H, n, dv, hdv, 0);
+            return launched();
+        });
+    if (s == ATTN_OK) g_last_launches = 4;
+    return s;
+}
+
 const char* attn_status_string(attn_status_t s) {
     switch (s) {
         case ATTN_OK: return "ok";

@@ -10,7 +10,9 @@
 //   dWq  = X^T A[:, 0:Hd], dWk, dWv likewise   (K runs over all B*n tokens:
 //                                               the batch sum of "Lesson 4",
 //                                               Step 4)
-// Both are plain 16-byte copies, bound by HBM bandwidth.
+// For the output projection of Problem 10 the same copy merges O into
+// [O_1 ... O_H] and tokens_to_heads slices G Wo^T back into per-head blocks.
+// All are plain 16-byte copies, bound by HBM bandwidth.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -53,6 +55,27 @@ concat_cols(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ d
         const size_t r = i / cc;
         const uint4 v = reinterpret_cast<const uint4*>(src)[i];
         *reinterpret_cast<uint4*>(dst + r * ld + col0 + 8 * c) = v;
+    }
+}
+
+// The inverse of heads_to_tokens: dst[((b*H + h)*n + t)*w + j] =
+// src[(b*n + t) * ld + col0 + h*w + j] (the column blocks of G Wo^T back into
+// per-head gradients, "Attention backward", Problem 10).
+__global__ void __launch_bounds__(kThreads)
+tokens_to_heads(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int B,
+                int H, int n, int w, int ld, int col0) {
+    const int cw = w / 8;
+    const size_t total = size_t(B) * H * n * cw;
+    for (size_t i = size_t(blockIdx.x) * kThreads + threadIdx.x; i < total;
+         i += size_t(gridDim.x) * kThreads) {
+        const int jc = int(i % cw);
+        size_t r = i / cw;
+        const int t = int(r % n);
+        r /= n;
+        const int h = int(r % H);
+        const int b = int(r / H);
+        reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<const uint4*>(
+            src + (size_t(b) * n + t) * ld + col0 + size_t(h) * w + 8 * jc);
     }
 }
 

@@ -146,3 +146,19 @@ def test_projection_workspace_formula(L):
         assert L.attn_proj_bwd_workspace_size(*args, 1) == expect(*args)
     assert L.attn_proj_bwd_workspace_size(2, 64, 64, 2, 64, 64, 0) == 0
     assert L.attn_proj_bwd_workspace_size(2, 64, 60, 2, 64, 64, 1) == 0
+
+
+def outproj(L, o=P, ws=P, wsb=1 << 40, B=2, n=64, d_model=64, H=2, dv=64, dt=1):
+    return L.lib.attn_outproj_bwd(o, P, P, P, P, ws, wsb, B, n, d_model, H, dv, dt, NUL)
+
+
+def test_argument_checks_output_projection(L):
+    assert outproj(L, o=NUL) == 1
+    assert outproj(L, H=0) == 2
+    assert outproj(L, dv=20) == 2
+    assert outproj(L, dt=0) == 4
+    assert outproj(L, o=MIS) == 5
+    assert outproj(L, wsb=16) == 6
+    r = lambda x: -(-x // 256) * 256
+    assert L.attn_outproj_bwd_workspace_size(2, 64, 64, 2, 64, 1) == 2 * r(2 * 64 * 2 * 64 * 2)
+    assert L.attn_outproj_bwd_workspace_size(2, 64, 64, 2, 64, 0) == 0

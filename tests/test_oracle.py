@@ -534,3 +534,68 @@ def test_projection_backward_mutants_fail(monkeypatch):
     monkeypatch.undo()
     dWq_good = ref.projection_backward(X, Wq, Wk, Wv, dQ, dK, dV)[1]
     assert np.max(np.abs(dWq_bad - dWq_good)) > 1e-3
+
+
+
+# --------------------------------------------------------------------------
+# Multi-head output projection (Problem 10)
+# --------------------------------------------------------------------------
+def test_output_projection_backward_finite_differences():
+    """dWo and every dO_h entry against central differences of
+    L = sum(Y * G), Y = [O_1 ... O_H] Wo, and dQ, dK, dV through attention with
+    dO = dO_h: the chain of Problem 10 into Problems 2-6."""
+    rng = np.random.default_rng(21)
+    B, H, n, d, dv, C = 2, 3, 4, 2, 3, 5
+    Q, K, V = (rng.standard_normal((B, H, n, w)) for w in (d, d, dv))
+    Wo = rng.standard_normal((H * dv, C)) * 0.5
+    G = rng.standard_normal((B, n, C))
+    O, _ = ref.attention_forward(Q, K, V, True)
+    dO, dWo = ref.output_projection_backward(O, Wo, G)
+    assert dO.shape == O.shape and dWo.shape == Wo.shape
+    eps = 1e-6
+
+    def loss_O(Ov):
+        return float(np.sum(ref.output_projection(Ov, Wo) * G))
+
+    def loss_W(W):
+        return float(np.sum(ref.output_projection(O, W) * G))
+
+    def loss_Q(Qv):
+        return float(np.sum(ref.output_projection(ref.attention_forward(Qv, K, V, True)[0], Wo) * G))
+
+    for f, p, want in ((loss_W, Wo, dWo), (loss_O, O, dO)):
+        num = np.zeros_like(p)
+        for idx in np.ndindex(p.shape):
+            orig = p[idx]
+            p[idx] = orig + eps
+            lp = f(p)
+            p[idx] = orig - eps
+            lm = f(p)
+            p[idx] = orig
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(want, num, rtol=1e-6, atol=1e-8)
+    dQ, _, _ = ref.attention_backward(Q, K, V, dO, True)
+    num = np.zeros_like(Q)
+    for idx in np.ndindex(Q.shape):
+        orig = Q[idx]
+        Q[idx] = orig + eps
+        lp = loss_Q(Q)
+        Q[idx] = orig - eps
+        lm = loss_Q(Q)
+        Q[idx] = orig
+        num[idx] = (lp - lm) / (2 * eps)
+    np.testing.assert_allclose(dQ, num, rtol=1e-5, atol=1e-8)
+
+
+def test_output_projection_backward_mutant_fails(monkeypatch):
+    """Slicing G Wo^T into the wrong head blocks (a transpose of the head and
+    width axes) fails the pin."""
+    rng = np.random.default_rng(22)
+    O = rng.standard_normal((1, 2, 3, 2))
+    Wo = rng.standard_normal((4, 3))
+    G = rng.standard_normal((1, 3, 3))
+    good, _ = ref.output_projection_backward(O, Wo, G)
+    monkeypatch.setattr(ref, "split_heads",
+                        lambda T, H: T.reshape(T.shape[0], T.shape[1], T.shape[2] // H, H).transpose(0, 3, 1, 2))
+    bad, _ = ref.output_projection_backward(O, Wo, G)
+    assert np.max(np.abs(bad - good)) > 1e-3

@@ -69,3 +69,23 @@ def test_projection_backward_after_attention():
                                    dQr, dKr, dVr)
     errs = {name: rel_err(to64(g_), w) for name, g_, w in zip(("dX", "dWq", "dWk", "dWv"), got, want)}
     assert all(v <= 3e-2 for v in errs.values()), errs
+
+
+@pytest.mark.parametrize("B,n,d_model,H,dv", [
+    (2, 200, 200, 3, 40),      # ragged everywhere
+    (1, 384, 512, 4, 128),
+    (2, 64, 8, 1, 8),
+])
+def test_output_projection_backward(B, n, d_model, H, dv):
+    g = torch.Generator().manual_seed(B + n + d_model)
+    O = torch.randn(B, H, n, dv, generator=g).to(torch.bfloat16)
+    Wo = (torch.randn(H * dv, d_model, generator=g) * (H * dv) ** -0.5).to(torch.bfloat16)
+    G = torch.randn(B, n, d_model, generator=g).to(torch.bfloat16)
+    dev = torch.device("cuda:0")
+    dO, dWo = lib.attn_outproj_bwd(O.to(dev), Wo.to(dev), G.to(dev))
+    torch.cuda.synchronize()
+    assert lib.attn_get_device_error() == 0
+    assert lib.attn_last_launch_count() == 4
+    want_dO, want_dWo = ref.output_projection_backward(*(t.to(torch.float64).numpy() for t in (O, Wo, G)))
+    errs = {"dO": rel_err(to64(dO), want_dO), "dWo": rel_err(to64(dWo), want_dWo)}
+    assert all(v <= TOL["bf16"] for v in errs.values()), errs
