@@ -381,9 +381,10 @@ attn_status_t gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* D, int M,
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn::gemmtc::kSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    dim3 grid((M + attn::gemmtc::kBM - 1) / attn::gemmtc::kBM,
-              (N + attn::gemmtc::kBN - 1) / attn::gemmtc::kBN);
-    if (grid.y > 65535) return ATTN_ERR_SHAPE;
+    const long long tiles = static_cast<long long>((M + attn::gemmtc::kBM - 1) / attn::gemmtc::kBM) *
+                            ((N + attn::gemmtc::kBN - 1) / attn::gemmtc::kBN);
+    if (tiles > 0x7fffffffll) return ATTN_ERR_SHAPE;
+    const dim3 grid(static_cast<unsigned>(tiles));
     return traced(ATTN_KERNEL_GEMM, st, [&] {
         kern<<<grid, attn::gemmtc::kThreads, attn::gemmtc::kSmemBytes, st>>>(
             ma, mb, static_cast<__nv_bfloat16*>(D), M, N, K, ldd, kWaitBudgetNs);

@@ -22,6 +22,7 @@ namespace attn {
 namespace gemmtc {
 
 constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kGroupM = 8;     // row tiles per rasterisation group
 constexpr int kThreads = 192;
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;          // 32 KB
@@ -48,7 +49,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     Bars* bars = reinterpret_cast<Bars*>(smem + kOffBar);
     volatile int* abort_flag = &bars->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = int(blockIdx.x) * kBM, n0 = int(blockIdx.y) * kBN;
+    // Tile order: groups of kGroupM row tiles, column tiles across each group,
+    // so the CTAs in flight share their A row panels and B column panels in L2.
+    const int mt = (M + kBM - 1) / kBM, nt = (N + kBN - 1) / kBN;
+    const int b = int(blockIdx.x);
+    const int group = b / (kGroupM * nt);
+    const int gm = min(kGroupM, mt - group * kGroupM);
+    const int within = b - group * kGroupM * nt;
+    const int m0 = (group * kGroupM + within % gm) * kBM, n0 = (within / gm) * kBN;
     const int num_kb = (K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
