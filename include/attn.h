@@ -33,8 +33,12 @@
  *    than ATTN_OK means that nothing was launched and no output was written.
  *    ATTN_ERR_CUDA reports a launch error from the CUDA runtime.
  *  - Kernel paths: bf16 with d == dv in {64, 128} runs on the tcgen05 tensor
- *    cores (TMA-fed, TMEM accumulators). f32, and bf16 of any other width up
- *    to 128, runs on a CUDA-core (FFMA) path in fp32 arithmetic.
+ *    cores (TMA-fed, TMEM accumulators). f32 with d, dv <= 64 (multiples of
+ *    4) also runs on the tensor cores, each fp32 operand split into three
+ *    bf16 pieces and each product taken as the six piece products that
+ *    reach fp32 precision (about 2^-25 relative per product). Other f32
+ *    shapes, and bf16 of any other width up to 128, run on a CUDA-core
+ *    (FFMA) path in fp32 arithmetic.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -60,8 +64,8 @@ typedef enum {
 typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype_t;
 
 /* Which kernels a call may use. ATTN_PATH_AUTO picks the tensor-core path
- * where it applies (bf16, d == dv in {64, 128}) and the CUDA-core path
- * otherwise. ATTN_PATH_SIMT forces the CUDA-core path. ATTN_PATH_TENSOR
+ * where it applies (bf16 with d == dv in {64, 128}; f32 with d, dv <= 64 and
+ * multiples of 4) and the CUDA-core path otherwise. ATTN_PATH_SIMT forces the CUDA-core path. ATTN_PATH_TENSOR
  * requires the tensor-core path and makes other shapes ATTN_ERR_UNSUPPORTED.
  * The setting is process-wide and applies to calls made after it. */
 typedef enum { ATTN_PATH_AUTO = 0, ATTN_PATH_SIMT = 1, ATTN_PATH_TENSOR = 2 } attn_path_t;
@@ -179,7 +183,10 @@ typedef enum {
     ATTN_KERNEL_BWD_SIMT = 5,     /* CUDA-core backward                       */
     ATTN_KERNEL_FINALIZE = 6,     /* dQ accumulator -> dQ                      */
     ATTN_KERNEL_PROJ_GATHER = 7,  /* per-head gradients / weights side by side */
-    ATTN_KERNEL_GEMM = 8          /* tcgen05 GEMM of the projection gradients  */
+    ATTN_KERNEL_GEMM = 8,         /* tcgen05 GEMM of the projection gradients  */
+    ATTN_KERNEL_FWD_F32X = 9,     /* tcgen05 forward, fp32 by bf16 pieces      */
+    ATTN_KERNEL_BWD_F32X_KV = 10, /* ... backward pass for dK, dV              */
+    ATTN_KERNEL_BWD_F32X_DQ = 11  /* ... backward pass for dQ                  */
 } attn_kernel_id_t;
 
 typedef struct {

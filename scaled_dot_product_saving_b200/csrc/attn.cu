@@ -20,6 +20,7 @@
 #include "bwd_tc.cuh"
 #include "gemm_tc.cuh"
 #include "proj.cuh"
+#include "f32x_tc.cuh"
 
 namespace {
 
@@ -45,16 +46,27 @@ attn_status_t check_sizes(int B, int H, int n, int m, int d, int dv, attn_dtype_
     return ATTN_OK;
 }
 
+enum class Path { kSimt, kTensorBf16, kTensorF32x };
+
 bool tensor_path_fits(attn_dtype_t dtype, int d, int dv) {
     return dtype == ATTN_BF16 && d == dv && (d == 64 || d == 128);
 }
 
-// Decide the path; ATTN_OK and *use_tensor set, or an error.
-attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, bool* use_tensor) {
+// fp32 on the tensor cores by bf16 pieces: widths padded to 64 columns,
+// 16-byte row loads.
+bool f32x_path_fits(attn_dtype_t dtype, int d, int dv) {
+    return dtype == ATTN_F32 && d <= attn::f32x::kWidth && dv <= attn::f32x::kWidth &&
+           d % 4 == 0 && dv % 4 == 0;
+}
+
+// Decide the path; ATTN_OK and *path set, or an error.
+attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, Path* path) {
     const int p = g_path.load();
-    const bool fits = tensor_path_fits(dtype, d, dv);
-    if (p == ATTN_PATH_TENSOR && !fits) return ATTN_ERR_UNSUPPORTED;
-    *use_tensor = fits && p != ATTN_PATH_SIMT;
+    const bool bf16 = tensor_path_fits(dtype, d, dv);
+    const bool f32x = f32x_path_fits(dtype, d, dv);
+    if (p == ATTN_PATH_TENSOR && !bf16 && !f32x) return ATTN_ERR_UNSUPPORTED;
+    if (p == ATTN_PATH_SIMT || (!bf16 && !f32x)) *path = Path::kSimt;
+    else *path = bf16 ? Path::kTensorBf16 : Path::kTensorF32x;
     return ATTN_OK;
 }
 
@@ -243,9 +255,9 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
 template <typename T>
 attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float* lse2, float* Dd,
                          float* dQacc, int* sched, int BH, int n, int n_pad, int d, int dv,
-                         float d_scale, cudaStream_t st) {
+                         float d_scale, bool zero_dq, cudaStream_t st) {
     const size_t rows = static_cast<size_t>(BH) * n_pad;
-    const size_t dq_elems = static_cast<size_t>(BH) * n * d;
+    const size_t dq_elems = zero_dq ? static_cast<size_t>(BH) * n * d : 0;
     const bool vec = sizeof(T) == 2 && dv % 8 == 0 && (dv / 8) <= 32 && 32 % (dv / 8) == 0 &&
                      dq_elems % 4 == 0;
     if (vec) {
@@ -325,6 +337,65 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
             mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, sched, n_pad, n, m, BH, head_group, causal, scale,
+            scale * kLog2e, kWaitBudgetNs);
+        return launched();
+    });
+}
+
+// fp32 by bf16 pieces: one CTA per (128-row tile, head), heads fastest.
+attn_status_t f32x_grid(int rows, int BH, unsigned* grid) {
+    const long long g = static_cast<long long>((rows + attn::f32x::kBig - 1) / attn::f32x::kBig) * BH;
+    if (g > 0x7fffffffll) return ATTN_ERR_SHAPE;
+    *grid = static_cast<unsigned>(g);
+    return ATTN_OK;
+}
+
+attn_status_t fwd_f32x(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH,
+                       int n, int m, int d, int dv, int causal, float scale, cudaStream_t st) {
+    namespace fx = attn::f32x;
+    unsigned grid = 0;
+    attn_status_t s = f32x_grid(n, BH, &grid);
+    if (s != ATTN_OK) return s;
+    if (cudaFuncSetAttribute(fx::fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fx::kFwdSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return traced(ATTN_KERNEL_FWD_F32X, st, [&] {
+        fx::fwd_kernel<<<grid, fx::kThreads, fx::kFwdSmemBytes, st>>>(
+            static_cast<const float*>(Q), static_cast<const float*>(K),
+            static_cast<const float*>(V), static_cast<float*>(O), LSE, n, m, d, dv, BH, causal,
+            scale * kLog2e, kWaitBudgetNs);
+        return launched();
+    });
+}
+
+attn_status_t bwd_f32x(const void* Q, const void* K, const void* V, const void* dO,
+                       const float* lse2, const float* Dd, int n_pad, void* dQ, void* dK, void* dV,
+                       int BH, int n, int m, int d, int dv, int causal, float scale,
+                       cudaStream_t st) {
+    namespace fx = attn::f32x;
+    unsigned grid_kv = 0, grid_dq = 0;
+    attn_status_t s = f32x_grid(m, BH, &grid_kv);
+    if (s == ATTN_OK) s = f32x_grid(n, BH, &grid_dq);
+    if (s != ATTN_OK) return s;
+    if (cudaFuncSetAttribute(fx::bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fx::kKvSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(fx::bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fx::kDqSmemBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const float* q = static_cast<const float*>(Q);
+    const float* k = static_cast<const float*>(K);
+    const float* v = static_cast<const float*>(V);
+    const float* g = static_cast<const float*>(dO);
+    s = traced(ATTN_KERNEL_BWD_F32X_KV, st, [&] {
+        fx::bwd_kv_kernel<<<grid_kv, fx::kBwdThreads, fx::kKvSmemBytes, st>>>(
+            q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dK), static_cast<float*>(dV), n, m,
+            d, dv, BH, causal, scale, scale * kLog2e, kWaitBudgetNs);
+        return launched();
+    });
+    if (s != ATTN_OK) return s;
+    return traced(ATTN_KERNEL_BWD_F32X_DQ, st, [&] {
+        fx::bwd_dq_kernel<<<grid_dq, fx::kBwdThreads, fx::kDqSmemBytes, st>>>(
+            q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dQ), n, m, d, dv, BH, causal, scale,
             scale * kLog2e, kWaitBudgetNs);
         return launched();
     });
@@ -417,11 +488,13 @@ attn_status_t attn_fwd(const void* Q, const void* K, const void* V, void* O, flo
     if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_NULL;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
         return ATTN_ERR_ALIGN;
-    bool tensor = false;
-    if ((s = choose_path(dtype, d, dv, &tensor)) != ATTN_OK) return s;
+    Path path = Path::kSimt;
+    if ((s = choose_path(dtype, d, dv, &path)) != ATTN_OK) return s;
     const int BH = B * H;
     cudaStream_t st = as_stream(stream);
-    if (tensor)
+    if (path == Path::kTensorF32x)
+        s = fwd_f32x(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+    else if (path == Path::kTensorBf16)
         s = (d == 64) ? fwd_tensor<64>(Q, K, V, O, LSE, BH, n, m, causal, scale, st)
                       : fwd_tensor<128>(Q, K, V, O, LSE, BH, n, m, causal, scale, st);
     else if (dtype == ATTN_F32)
@@ -446,8 +519,9 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     const Workspace w = carve(B, H, n, d);
     if (!workspace || workspace_bytes < w.total) return ATTN_ERR_WORKSPACE;
     if (!aligned16(workspace)) return ATTN_ERR_ALIGN;
-    bool tensor = false;
-    if ((s = choose_path(dtype, d, dv, &tensor)) != ATTN_OK) return s;
+    Path path = Path::kSimt;
+    if ((s = choose_path(dtype, d, dv, &path)) != ATTN_OK) return s;
+    const bool tensor = path != Path::kSimt;
 
     const int BH = B * H;
     cudaStream_t st = as_stream(stream);
@@ -458,15 +532,20 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     int* sched = reinterpret_cast<int*>(ws + w.sched_off);
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
 
-    // The tensor-core backward takes D already multiplied by the scale.
+    // The tensor-core backwards take D already multiplied by the scale; the
+    // fp32 one writes dQ directly and needs no zeroed accumulator.
     const float d_scale = tensor ? scale : 1.0f;
+    const bool zero_dq = path != Path::kTensorF32x;
     s = (dtype == ATTN_F32)
             ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv, d_scale,
-                                st)
+                                zero_dq, st)
             : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv,
-                                        d_scale, st);
+                                        d_scale, zero_dq, st);
     if (s != ATTN_OK) return s;
-    if (tensor) {
+    if (path == Path::kTensorF32x) {
+        s = bwd_f32x(Q, K, V, dO, lse2, Dd, w.n_pad, dQ, dK, dV, BH, n, m, d, dv, causal, scale,
+                     st);
+    } else if (path == Path::kTensorBf16) {
         s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
                                        n, m, causal, scale, st)
                       : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,

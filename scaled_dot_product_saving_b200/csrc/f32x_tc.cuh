@@ -1,0 +1,693 @@
+// f32x_tc.cuh -- fp32 attention forward and backward on the tensor cores, by
+// splitting every fp32 operand into three bf16 pieces.
+//
+// The arithmetic is that of "Attention Backward Pass (dQ, dK, dV) -
+// Transformer Architecture", sections "Forward" and "Backward", as in the
+// bf16 kernels: S = scale Q K^T, P = softmax(S) (causal: key j > query i
+// masked), O = P V, and with D = rowsum(dO * O) ("Attention Backpropagation:
+// Step by step derivation", section "Gradient of S"): dV = P^T dO,
+// dS = P * (dO V^T - D), dQ = scale dS K, dK = scale dS^T Q.
+//
+// Precision. A value x in fp32 is written as x0 + x1 + x2 with
+//   x0 = bf16(x),  x1 = bf16(x - x0),  x2 = bf16(x - x0 - x1)
+// (both subtractions are exact in fp32), which leaves |x - x0 - x1 - x2| at
+// most about 2^-26 |x|. A product a b is the sum of the six piece products
+// a_i b_j with i + j <= 2; the three left out are below about 2^-25 |a b|
+// together. Each piece product is one bf16 tcgen05 MMA accumulating in fp32
+// in TMEM, so one fp32 contraction costs six bf16 MMAs -- the tensor time of
+// three tf32 MMAs (tf32 runs at half the bf16 rate), with operands rounded to
+// 24 significant bits instead of the 22 of a tf32 hi/lo pair, and with the
+// operand layouts of the bf16 kernels.
+//
+// Shapes. Operands are zero-padded to 64 columns, so d, dv <= 64 (multiples
+// of 4 for 16-byte loads). Every MMA is M = 128, N = 64, K = 16: the 128 rows
+// a CTA owns sit one per thread and TMEM lane, the streamed tiles have 64
+// rows. Pieces of a tile are stored one after another, each in the 128-byte
+// swizzled layout the MMA descriptors read (rows of 64 bf16).
+//
+// Kernels (128 threads, one elected thread issues the MMAs, all threads load,
+// split and run the elementwise steps):
+//   fwd_kernel     a 128-query tile, 64-key tiles: S (SS), online softmax in
+//                  registers, P split into TMEM, P V (TS) added into O in
+//                  registers with the running rescale.
+//   bwd_kv_kernel  a 128-key tile, 64-query tiles: S^T, dP^T (SS), P^T and
+//                  dS^T split into TMEM, dV += P^T dO and dK += dS^T Q (TS).
+//   bwd_dq_kernel  a 128-query tile, 64-key tiles: S, dP (SS), dS split into
+//                  TMEM, dQ += dS K (TS). dQ is written once, no atomics.
+// The backward is two passes that each recompute S and dP, so that neither
+// needs a transposed copy of dS in shared memory (three pieces of a 128 x 128
+// tile would not fit beside the operands). Streamed tiles are double
+// buffered: the loads of tile t + 2 run while the MMAs of tile t + 1 do.
+//
+// The backward takes D multiplied by the scale and the LSE in base 2, from
+// the preprocess kernel (padded to whole 128-row tiles: LSE = +inf and D = 0
+// in the padding, so padded query rows get P = 0).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+namespace f32x {
+
+constexpr int kThreads = 128;
+constexpr int kBig = 128;                       // rows a CTA owns (= threads = TMEM lanes)
+constexpr int kSmall = 64;                      // rows of a streamed tile
+constexpr int kWidth = 64;                      // padded operand width
+constexpr int kBigPiece = kBig * 128;           // one bf16 piece of a 128 x 64 tile
+constexpr int kSmallPiece = kSmall * 128;       // one bf16 piece of a 64 x 64 tile
+constexpr int kBigTile = 3 * kBigPiece;         // 48 KB
+constexpr int kSmallTile = 3 * kSmallPiece;     // 24 KB
+constexpr float kLn2 = 0.6931471805599453f;
+
+// The six piece pairs (a, b) with a + b <= 2, smallest products first.
+__host__ __device__ constexpr int pair_a(int p) { return p == 0 ? 2 : p == 1 ? 1 : p == 2 ? 0 : p == 3 ? 1 : 0; }
+__host__ __device__ constexpr int pair_b(int p) { return p == 0 ? 0 : p == 1 ? 1 : p == 2 ? 2 : p == 3 ? 0 : p == 4 ? 1 : 0; }
+
+struct Bars {
+    uint64_t bar_a;       // first MMA group of a step has completed
+    uint64_t bar_b;       // second MMA group of a step has completed
+    uint64_t drain;       // every MMA of the CTA has completed (teardown)
+    uint32_t tmem_base;
+};
+
+// ------------------------------------------------------------ splitting
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) {
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Two fp32 values (x: lower element) into their three bf16 pieces, packed
+// two to a word.
+__device__ __forceinline__ void split2(float x, float y, uint32_t& w0, uint32_t& w1, uint32_t& w2) {
+    const __nv_bfloat162 h0 = __floats2bfloat162_rn(x, y);
+    const float2 f0 = __bfloat1622float2(h0);
+    const float rx = __fsub_rn(x, f0.x), ry = __fsub_rn(y, f0.y);
+    const __nv_bfloat162 h1 = __floats2bfloat162_rn(rx, ry);
+    const float2 f1 = __bfloat1622float2(h1);
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fsub_rn(rx, f1.x), __fsub_rn(ry, f1.y));
+    w0 = bf2_bits(h0);
+    w1 = bf2_bits(h1);
+    w2 = bf2_bits(h2);
+}
+
+// Rows [row0, row0 + R) of a row-major [rows_valid, width] fp32 matrix into
+// the three pieces at `dst` (R * 128 bytes apart), 128-byte swizzled rows of
+// 64 bf16. Rows at or past rows_valid and columns at or past width are zero.
+// width % 4 == 0; the matrix starts 16-byte aligned.
+template <int R, int NT>
+__device__ __forceinline__ void load_split(const float* __restrict__ src, int row0, int rows_valid,
+                                           int width, uint8_t* dst, int tid) {
+#pragma unroll 2
+    for (int k = tid; k < R * 8; k += NT) {
+        const int r = k >> 3, c = k & 7;
+        const int grow = row0 + r, col = 8 * c;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+        if (grow < rows_valid && col < width) {
+            const float4* p = reinterpret_cast<const float4*>(src + size_t(grow) * width + col);
+            a = __ldg(p);
+            if (col + 8 <= width) b = __ldg(p + 1);
+        }
+        uint4 p0, p1, p2;
+        split2(a.x, a.y, p0.x, p1.x, p2.x);
+        split2(a.z, a.w, p0.y, p1.y, p2.y);
+        split2(b.x, b.y, p0.z, p1.z, p2.z);
+        split2(b.z, b.w, p0.w, p1.w, p2.w);
+        const int off = r * 128 + ((c ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst + off) = p0;
+        *reinterpret_cast<uint4*>(dst + R * 128 + off) = p1;
+        *reinterpret_cast<uint4*>(dst + 2 * R * 128 + off) = p2;
+    }
+}
+
+// 32 values of this thread's row into the three pieces in TMEM: piece a of
+// the 64-wide row at columns col + 32 a .. +31 (two bf16 per column), this
+// half (h = 0, 1) at +16 h.
+__device__ __forceinline__ void split_to_tmem(const float (&v)[32], uint32_t taddr) {
+    uint32_t w0[16], w1[16], w2[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) split2(v[2 * e], v[2 * e + 1], w0[e], w1[e], w2[e]);
+    tmem_st16(taddr, w0);
+    tmem_st16(taddr + 32, w1);
+    tmem_st16(taddr + 64, w2);
+}
+
+// ------------------------------------------------------------ MMA groups
+// D (+)= sum over the six pairs of A_a B_b^T, K = 64. A: 128 rows, K-major,
+// pieces a_stride bytes apart; B: 64 rows, K-major, pieces b_stride apart.
+__device__ __forceinline__ void mma6_ss(uint32_t d, uint32_t sa, uint32_t a_stride, uint32_t sb,
+                                        uint32_t b_stride, uint32_t idesc) {
+#pragma unroll
+    for (int p = 0; p < 6; ++p)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_ss(d, sdesc_sw128(sa + pair_a(p) * a_stride + kk * 32, 16, 1024),
+                   sdesc_sw128(sb + pair_b(p) * b_stride + kk * 32, 16, 1024), idesc,
+                   (p > 0 || kk > 0) ? 1u : 0u);
+}
+
+// D (+)= sum over the six pairs of A_a B_b, K = 64. A in TMEM (pieces 32
+// columns apart, 8 columns per 16-deep step); B in shared memory, MN-major:
+// 64 rows along K, 64 columns along N, pieces kSmallPiece apart.
+__device__ __forceinline__ void mma6_ts(uint32_t d, uint32_t ta, uint32_t sb, uint32_t idesc,
+                                        bool accumulate) {
+#pragma unroll
+    for (int p = 0; p < 6; ++p)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_ts(d, ta + 32 * pair_a(p) + 8 * kk,
+                   sdesc_sw128(sb + pair_b(p) * kSmallPiece + kk * 2048, kSmallPiece, 1024), idesc,
+                   (accumulate || p > 0 || kk > 0) ? 1u : 0u);
+}
+
+constexpr uint32_t kIdSS = idesc_bf16_f32(128, 64, 0, 0);   // both K-major
+constexpr uint32_t kIdTS = idesc_bf16_f32(128, 64, 0, 1);   // B MN-major
+
+// Common prologue / epilogue pieces.
+__device__ __forceinline__ void init_bars(Bars* bars, uint32_t tmem_cols) {
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->bar_a, 1);
+        mbar_init(&bars->bar_b, 1);
+        mbar_init(&bars->drain, 1);
+        fence_mbar_init();
+    }
+    if ((threadIdx.x >> 5) == 0) {
+        tmem_alloc(&bars->tmem_base, tmem_cols);
+        tmem_relinquish();
+    }
+}
+
+// Wait until every MMA issued by thread 0 has completed, then free TMEM.
+__device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem, uint32_t tmem_cols,
+                                         uint64_t budget_ns) {
+    if (threadIdx.x == 0) {
+        mma_commit(&bars->drain);
+        if (!mbar_wait_timed(&bars->drain, 0, budget_ns)) record_device_error(kErrTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tmem_cols);
+    }
+}
+
+// Load 64 fp32 columns of this thread's TMEM lane at `taddr` (two 32-column
+// loads) into v.
+__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
+    uint32_t a[32], b[32];
+    tmem_ld32(taddr, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld_wait(a);
+    tmem_ld_wait(b);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        v[c] = __uint_as_float(a[c]);
+        v[32 + c] = __uint_as_float(b[c]);
+    }
+}
+
+// Store columns [0, width) of a 64-wide fp32 row (width % 4 == 0).
+__device__ __forceinline__ void store_row(float* dst, const float (&v)[64], int width, float mul) {
+#pragma unroll
+    for (int c = 0; c < 64; c += 4)
+        if (c < width)
+            *reinterpret_cast<float4*>(dst + c) =
+                make_float4(v[c] * mul, v[c + 1] * mul, v[c + 2] * mul, v[c + 3] * mul);
+}
+
+// ================================================================ forward
+// TMEM columns: S (64), P V of the current key tile (64), P pieces (96).
+constexpr uint32_t kFwdColS = 0, kFwdColPV = 64, kFwdColP = 128, kFwdTmemCols = 256;
+constexpr int kFwdOffQ = 0;
+constexpr int kFwdOffK = kFwdOffQ + kBigTile;          // two buffers
+constexpr int kFwdOffV = kFwdOffK + 2 * kSmallTile;    // two buffers
+constexpr int kFwdOffBar = kFwdOffV + 2 * kSmallTile;
+constexpr int kFwdSmemBytes = kFwdOffBar + 128;
+
+// Grid: one CTA per (128-query tile, head), heads fastest; causal grids start
+// with the last query tiles (the most key tiles).
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+           float* __restrict__ O, float* __restrict__ LSE, int n, int m, int d, int dv, int BH,
+           int causal, float scale_log2, unsigned long long budget_ns) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    Bars* bars = reinterpret_cast<Bars*>(smem + kFwdOffBar);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int num_qt = (n + kBig - 1) / kBig;
+    const int bh = int(blockIdx.x % unsigned(BH));
+    const int rank = int(blockIdx.x / unsigned(BH));
+    const int qt = causal ? num_qt - 1 - rank : rank;
+    const int q0 = qt * kBig, row = q0 + tid;
+    const float* Qh = Q + size_t(bh) * n * d;
+    const float* Kh = K + size_t(bh) * m * d;
+    const float* Vh = V + size_t(bh) * m * dv;
+    const int nkt = (m + kSmall - 1) / kSmall;
+    const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
+
+    init_bars(bars, kFwdTmemCols);
+    const bool aligned = (smem_addr(smem) & 1023u) == 0;
+    if (aligned) {
+        load_split<kBig, kThreads>(Qh, q0, n, d, smem + kFwdOffQ, tid);
+        load_split<kSmall, kThreads>(Kh, 0, m, d, smem + kFwdOffK, tid);
+        load_split<kSmall, kThreads>(Vh, 0, m, dv, smem + kFwdOffV, tid);
+        if (T > 1) {
+            load_split<kSmall, kThreads>(Kh, kSmall, m, d, smem + kFwdOffK + kSmallTile, tid);
+            load_split<kSmall, kThreads>(Vh, kSmall, m, dv, smem + kFwdOffV + kSmallTile, tid);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t sQ = smem_addr(smem + kFwdOffQ);
+    const uint32_t sK = smem_addr(smem + kFwdOffK), sV = smem_addr(smem + kFwdOffV);
+    const int never = 0;
+
+    bool ok = aligned;
+    if (!aligned && tid == 0) record_device_error(kErrTimeout);
+    if (ok && tid == 0) {
+        mma6_ss(tmem + kFwdColS, sQ, kBigPiece, sK, kSmallPiece, kIdSS);
+        mma_commit(&bars->bar_a);
+    }
+    float o[64];
+#pragma unroll
+    for (int c = 0; c < 64; ++c) o[c] = 0.f;
+    float mrow = -INFINITY, lrow = 0.f;
+
+    for (int j = 0; ok && j < T; ++j) {
+        const int buf = j & 1;
+        float alpha = 1.f;
+        const bool got = mbar_wait_warp(&bars->bar_a, j & 1, &never, budget_ns);
+        if (got) {
+            tc_fence_after();
+            float s[64];
+            tmem_row64(tl + kFwdColS, s);
+            const int kb = j * kSmall;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                const int key = kb + c;
+                float x = s[c] * scale_log2;
+                if (key >= m || (causal && key > row)) x = -INFINITY;
+                s[c] = x;
+                mx = fmaxf(mx, x);
+            }
+            const float mnew = fmaxf(mrow, mx);
+            const float base = (mnew == -INFINITY) ? 0.f : mnew;
+            alpha = (mrow == -INFINITY) ? 0.f : ex2(mrow - base);
+            float lsum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                s[c] = ex2(s[c] - base);
+                lsum += s[c];
+            }
+            lrow = lrow * alpha + lsum;
+            mrow = mnew;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float v[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) v[c] = s[32 * h + c];
+                split_to_tmem(v, tl + kFwdColP + 16 * h);
+            }
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            break;
+        }
+        if (tid == 0) {
+            tc_fence_after();
+            mma6_ts(tmem + kFwdColPV, tmem + kFwdColP, sV + buf * kSmallTile, kIdTS, false);
+            mma_commit(&bars->bar_b);
+            if (j + 1 < T) {
+                mma6_ss(tmem + kFwdColS, sQ, kBigPiece, sK + (buf ^ 1) * kSmallTile, kSmallPiece,
+                        kIdSS);
+                mma_commit(&bars->bar_a);
+            }
+        }
+        const bool got2 = mbar_wait_warp(&bars->bar_b, j & 1, &never, budget_ns);
+        if (got2) {
+            tc_fence_after();
+            float pv[64];
+            tmem_row64(tl + kFwdColPV, pv);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) o[c] = fmaf(o[c], alpha, pv[c]);
+            // K_j (read by S_j) and V_j (read by P_j V_j) are free: tile j + 2.
+            if (j + 2 < T) {
+                load_split<kSmall, kThreads>(Kh, (j + 2) * kSmall, m, d, smem + kFwdOffK + buf * kSmallTile, tid);
+                load_split<kSmall, kThreads>(Vh, (j + 2) * kSmall, m, dv, smem + kFwdOffV + buf * kSmallTile, tid);
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got2)) {
+            ok = false;
+            break;
+        }
+    }
+
+    if (ok) {
+        if (row < n) {
+            store_row(O + (size_t(bh) * n + row) * dv, o, dv, 1.0f / lrow);
+            LSE[size_t(bh) * n + row] = (mrow + log2f(lrow)) * kLn2;
+        }
+    } else if (tid == 0) {
+        record_device_error(kErrTimeout);
+    }
+    teardown(bars, tmem, kFwdTmemCols, budget_ns);
+}
+
+// ================================================================ backward
+// Both backward kernels run two warpgroups (256 threads): thread t owns TMEM
+// lane / tile row t % 128 and the column half t / 128 of every 64-wide row,
+// so the elementwise work and the running sums are split between them.
+//
+// Accumulation. The tensor cores' fp32 accumulation is not rounded to
+// nearest: adding several hundred MMA steps into one TMEM accumulator (a
+// head of 1024 queries gives 16 tiles x 24 steps) drifts by about 1e-5 of
+// the result. So the MMAs of one streamed tile start a fresh partial sum in
+// TMEM (24 steps), and the threads add the partials into registers with
+// ordinary round-to-nearest fp32 adds.
+constexpr int kBwdThreads = 256;
+
+// 32 values into the three pieces in TMEM at taddr (piece a at +32 a), 16
+// values (8 columns) at a time.
+__device__ __forceinline__ void split32_to_tmem(const uint32_t (&v)[32], uint32_t taddr) {
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+        uint32_t w0[8], w1[8], w2[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            split2(__uint_as_float(v[16 * qq + 2 * e]), __uint_as_float(v[16 * qq + 2 * e + 1]),
+                   w0[e], w1[e], w2[e]);
+        tmem_st8(taddr + 8 * qq, w0);
+        tmem_st8(taddr + 8 * qq + 32, w1);
+        tmem_st8(taddr + 8 * qq + 64, w2);
+    }
+}
+
+// acc[0..31] += the 32 fp32 columns of this lane at taddr.
+__device__ __forceinline__ void add_tmem32(uint32_t taddr, float (&acc)[32]) {
+    uint32_t r[32];
+    tmem_ld32(taddr, r);
+    tmem_ld_wait(r);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] += __uint_as_float(r[c]);
+}
+
+// Columns [c0, c0 + 32) of a row, clipped to width (width, c0 multiples of 4).
+__device__ __forceinline__ void store_half(float* row, int c0, const float (&v)[32], int width) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4)
+        if (c0 + c < width)
+            *reinterpret_cast<float4*>(row + c0 + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+}
+
+// ---------------------------------------------------- dK and dV pass
+// TMEM columns: S^T (64), dP^T (64), this tile's dV (64) and dK (64), P^T
+// pieces (96), dS^T pieces (96).
+constexpr uint32_t kKvColS = 0, kKvColdP = 64, kKvColdV = 128, kKvColdK = 192, kKvColP = 256,
+                   kKvColdS = 352, kKvTmemCols = 512;
+constexpr int kKvOffK = 0;
+constexpr int kKvOffV = kKvOffK + kBigTile;
+constexpr int kKvOffQ = kKvOffV + kBigTile;            // two buffers
+constexpr int kKvOffdO = kKvOffQ + 2 * kSmallTile;     // two buffers
+constexpr int kKvOffRow = kKvOffdO + 2 * kSmallTile;   // [2][LSE 64 | D 64] floats
+constexpr int kKvOffBar = kKvOffRow + 4 * kSmall * 4;
+constexpr int kKvSmemBytes = kKvOffBar + 128;
+
+// Grid: one CTA per (128-key tile, head), heads fastest; causal grids start
+// with the first key tiles (the most query tiles).
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+              const float* __restrict__ dO, const float* __restrict__ lse2,
+              const float* __restrict__ Dd, int n_pad, float* __restrict__ dK,
+              float* __restrict__ dV, int n, int m, int d, int dv, int BH, int causal, float scale,
+              float scale_log2, unsigned long long budget_ns) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    Bars* bars = reinterpret_cast<Bars*>(smem + kKvOffBar);
+    float* sRow = reinterpret_cast<float*>(smem + kKvOffRow);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane128 = tid & 127, half = tid >> 7;
+    const int bh = int(blockIdx.x % unsigned(BH));
+    const int kt = int(blockIdx.x / unsigned(BH));
+    const int k0 = kt * kBig, krow = k0 + lane128;
+    const float* Qh = Q + size_t(bh) * n * d;
+    const float* Kh = K + size_t(bh) * m * d;
+    const float* Vh = V + size_t(bh) * m * dv;
+    const float* dOh = dO + size_t(bh) * n * dv;
+    const float* L2h = lse2 + size_t(bh) * n_pad;
+    const float* Dh = Dd + size_t(bh) * n_pad;
+    const int nqs = (n + kSmall - 1) / kSmall;
+    const int i0 = causal ? k0 / kSmall : 0;
+    const int T = nqs - i0;            // >= 1: causal has n == m > k0
+
+    auto load_q = [&](int idx, int buf) {
+        const int r0 = (i0 + idx) * kSmall;
+        load_split<kSmall, kBwdThreads>(Qh, r0, n, d, smem + kKvOffQ + buf * kSmallTile, tid);
+        load_split<kSmall, kBwdThreads>(dOh, r0, n, dv, smem + kKvOffdO + buf * kSmallTile, tid);
+        // rows < n_pad: 64-row tiles never pass the 128-row padding
+        if (tid < kSmall) sRow[buf * 128 + tid] = L2h[r0 + tid];
+        else if (tid < 2 * kSmall) sRow[buf * 128 + tid] = Dh[r0 + tid - kSmall];
+    };
+
+    init_bars(bars, kKvTmemCols);
+    const bool aligned = (smem_addr(smem) & 1023u) == 0;
+    if (aligned) {
+        load_split<kBig, kBwdThreads>(Kh, k0, m, d, smem + kKvOffK, tid);
+        load_split<kBig, kBwdThreads>(Vh, k0, m, dv, smem + kKvOffV, tid);
+        load_q(0, 0);
+        if (T > 1) load_q(1, 1);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16) + 32 * half;
+    const uint32_t sK = smem_addr(smem + kKvOffK), sV = smem_addr(smem + kKvOffV);
+    const uint32_t sQ = smem_addr(smem + kKvOffQ), sdO = smem_addr(smem + kKvOffdO);
+    const int never = 0;
+
+    bool ok = aligned;
+    if (!aligned && tid == 0) record_device_error(kErrTimeout);
+    if (ok && tid == 0) {
+        mma6_ss(tmem + kKvColS, sK, kBigPiece, sQ, kSmallPiece, kIdSS);
+        mma6_ss(tmem + kKvColdP, sV, kBigPiece, sdO, kSmallPiece, kIdSS);
+        mma_commit(&bars->bar_a);
+    }
+    float acc_v[32], acc_k[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc_v[c] = acc_k[c] = 0.f;
+
+    for (int idx = 0; ok && idx < T; ++idx) {
+        const int buf = idx & 1;
+        const int qb = (i0 + idx) * kSmall + 32 * half;     // first query of this half
+        const bool got = mbar_wait_warp(&bars->bar_a, idx & 1, &never, budget_ns);
+        if (got) {
+            tc_fence_after();
+            const float* Lrow = sRow + buf * 128 + 32 * half;
+            const float* Drow = Lrow + kSmall;
+            uint32_t sr[32], pr[32];
+            tmem_ld32(tl + kKvColS, sr);
+            tmem_ld32(tl + kKvColdP, pr);
+            tmem_ld_wait(sr);
+            tmem_ld_wait(pr);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -Lrow[c]));
+                if (causal && krow > qb + c) pv = 0.f;
+                sr[c] = __float_as_uint(pv);
+                pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -Drow[c]));
+            }
+            // this half's 32 queries are K elements 32 half .. +31: columns 16 half ..
+            split32_to_tmem(sr, tl - 32 * half + kKvColP + 16 * half);
+            split32_to_tmem(pr, tl - 32 * half + kKvColdS + 16 * half);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            break;
+        }
+        if (tid == 0) {
+            tc_fence_after();
+            mma6_ts(tmem + kKvColdV, tmem + kKvColP, sdO + buf * kSmallTile, kIdTS, false);
+            mma6_ts(tmem + kKvColdK, tmem + kKvColdS, sQ + buf * kSmallTile, kIdTS, false);
+            mma_commit(&bars->bar_b);
+            if (idx + 1 < T) {
+                mma6_ss(tmem + kKvColS, sK, kBigPiece, sQ + (buf ^ 1) * kSmallTile, kSmallPiece,
+                        kIdSS);
+                mma6_ss(tmem + kKvColdP, sV, kBigPiece, sdO + (buf ^ 1) * kSmallTile, kSmallPiece,
+                        kIdSS);
+                mma_commit(&bars->bar_a);
+            }
+        }
+        const bool got2 = mbar_wait_warp(&bars->bar_b, idx & 1, &never, budget_ns);
+        if (got2) {
+            tc_fence_after();
+            add_tmem32(tl + kKvColdV, acc_v);
+            add_tmem32(tl + kKvColdK, acc_k);
+            // Q_i, dO_i, their LSE and D are free once dV, dK of this tile are done.
+            if (idx + 2 < T) {
+                load_q(idx + 2, buf);
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got2)) {
+            ok = false;
+            break;
+        }
+    }
+
+    if (ok) {
+        if (krow < m) {
+            store_half(dV + (size_t(bh) * m + krow) * dv, 32 * half, acc_v, dv);
+            store_half(dK + (size_t(bh) * m + krow) * d, 32 * half, acc_k, d);
+        }
+    } else if (tid == 0) {
+        record_device_error(kErrTimeout);
+    }
+    teardown(bars, tmem, kKvTmemCols, budget_ns);
+}
+
+// ----------------------------------------------------------- dQ pass
+// TMEM columns: S (64), dP (64), this tile's dQ (64), dS pieces (96).
+constexpr uint32_t kDqColS = 0, kDqColdP = 64, kDqColdQ = 128, kDqColdS = 192, kDqTmemCols = 512;
+constexpr int kDqOffQ = 0;
+constexpr int kDqOffdO = kDqOffQ + kBigTile;
+constexpr int kDqOffK = kDqOffdO + kBigTile;           // two buffers
+constexpr int kDqOffV = kDqOffK + 2 * kSmallTile;      // two buffers
+constexpr int kDqOffBar = kDqOffV + 2 * kSmallTile;
+constexpr int kDqSmemBytes = kDqOffBar + 128;
+
+// Grid as the forward's.
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+              const float* __restrict__ dO, const float* __restrict__ lse2,
+              const float* __restrict__ Dd, int n_pad, float* __restrict__ dQ, int n, int m, int d,
+              int dv, int BH, int causal, float scale, float scale_log2,
+              unsigned long long budget_ns) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    Bars* bars = reinterpret_cast<Bars*>(smem + kDqOffBar);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane128 = tid & 127, half = tid >> 7;
+    const int num_qt = (n + kBig - 1) / kBig;
+    const int bh = int(blockIdx.x % unsigned(BH));
+    const int rank = int(blockIdx.x / unsigned(BH));
+    const int qt = causal ? num_qt - 1 - rank : rank;
+    const int q0 = qt * kBig, row = q0 + lane128;
+    const float* Qh = Q + size_t(bh) * n * d;
+    const float* Kh = K + size_t(bh) * m * d;
+    const float* Vh = V + size_t(bh) * m * dv;
+    const float* dOh = dO + size_t(bh) * n * dv;
+    const float l2 = lse2[size_t(bh) * n_pad + row];     // row < n_pad
+    const float dd = Dd[size_t(bh) * n_pad + row];
+    const int nkt = (m + kSmall - 1) / kSmall;
+    const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
+
+    init_bars(bars, kDqTmemCols);
+    const bool aligned = (smem_addr(smem) & 1023u) == 0;
+    if (aligned) {
+        load_split<kBig, kBwdThreads>(Qh, q0, n, d, smem + kDqOffQ, tid);
+        load_split<kBig, kBwdThreads>(dOh, q0, n, dv, smem + kDqOffdO, tid);
+        load_split<kSmall, kBwdThreads>(Kh, 0, m, d, smem + kDqOffK, tid);
+        load_split<kSmall, kBwdThreads>(Vh, 0, m, dv, smem + kDqOffV, tid);
+        if (T > 1) {
+            load_split<kSmall, kBwdThreads>(Kh, kSmall, m, d, smem + kDqOffK + kSmallTile, tid);
+            load_split<kSmall, kBwdThreads>(Vh, kSmall, m, dv, smem + kDqOffV + kSmallTile, tid);
+        }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    const uint32_t tl = tmem + (uint32_t((warp & 3) * 32) << 16) + 32 * half;
+    const uint32_t sQ = smem_addr(smem + kDqOffQ), sdO = smem_addr(smem + kDqOffdO);
+    const uint32_t sK = smem_addr(smem + kDqOffK), sV = smem_addr(smem + kDqOffV);
+    const int never = 0;
+
+    bool ok = aligned;
+    if (!aligned && tid == 0) record_device_error(kErrTimeout);
+    if (ok && tid == 0) {
+        mma6_ss(tmem + kDqColS, sQ, kBigPiece, sK, kSmallPiece, kIdSS);
+        mma6_ss(tmem + kDqColdP, sdO, kBigPiece, sV, kSmallPiece, kIdSS);
+        mma_commit(&bars->bar_a);
+    }
+    float acc[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c] = 0.f;
+
+    for (int j = 0; ok && j < T; ++j) {
+        const int buf = j & 1;
+        const int kb = j * kSmall + 32 * half;               // first key of this half
+        const bool got = mbar_wait_warp(&bars->bar_a, j & 1, &never, budget_ns);
+        if (got) {
+            tc_fence_after();
+            uint32_t sr[32], pr[32];
+            tmem_ld32(tl + kDqColS, sr);
+            tmem_ld32(tl + kDqColdP, pr);
+            tmem_ld_wait(sr);
+            tmem_ld_wait(pr);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                const int key = kb + c;
+                float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -l2));
+                if (key >= m || (causal && key > row)) pv = 0.f;
+                pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -dd));
+            }
+            split32_to_tmem(pr, tl - 32 * half + kDqColdS + 16 * half);
+            tmem_st_wait();
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            break;
+        }
+        if (tid == 0) {
+            tc_fence_after();
+            mma6_ts(tmem + kDqColdQ, tmem + kDqColdS, sK + buf * kSmallTile, kIdTS, false);
+            mma_commit(&bars->bar_b);
+            if (j + 1 < T) {
+                mma6_ss(tmem + kDqColS, sQ, kBigPiece, sK + (buf ^ 1) * kSmallTile, kSmallPiece,
+                        kIdSS);
+                mma6_ss(tmem + kDqColdP, sdO, kBigPiece, sV + (buf ^ 1) * kSmallTile, kSmallPiece,
+                        kIdSS);
+                mma_commit(&bars->bar_a);
+            }
+        }
+        const bool got2 = mbar_wait_warp(&bars->bar_b, j & 1, &never, budget_ns);
+        if (got2) {
+            tc_fence_after();
+            add_tmem32(tl + kDqColdQ, acc);
+            // K_j (read by S_j and dS_j K_j) and V_j (read by dP_j) are free.
+            if (j + 2 < T) {
+                load_split<kSmall, kBwdThreads>(Kh, (j + 2) * kSmall, m, d,
+                                                smem + kDqOffK + buf * kSmallTile, tid);
+                load_split<kSmall, kBwdThreads>(Vh, (j + 2) * kSmall, m, dv,
+                                                smem + kDqOffV + buf * kSmallTile, tid);
+                fence_proxy_async_smem();
+            }
+        }
+        tc_fence_before();
+        if (__syncthreads_or(!got2)) {
+            ok = false;
+            break;
+        }
+    }
+
+    if (ok) {
+        if (row < n) store_half(dQ + (size_t(bh) * n + row) * d, 32 * half, acc, d);
+    } else if (tid == 0) {
+        record_device_error(kErrTimeout);
+    }
+    teardown(bars, tmem, kDqTmemCols, budget_ns);
+}
+
+}  // namespace f32x
+}  // namespace attn

@@ -66,6 +66,9 @@ WORKLOADS = {
         "cross_b8h16_n512_m2048_d64", 8, 16, 512, 2048, 64, 64, "bf16", False, 4,
         std_qk=3.0, std_vo=1.0,
         doc="cross-attention B=8 H=16 n=512 m=2048 d=64 bf16, Q,K ~ N(0,9)"),
+    "causal_b4h16_n1024_d64_f32": Workload(
+        "causal_b4h16_n1024_d64_f32", 4, 16, 1024, 1024, 64, 64, "f32", True, 6,
+        doc="B=4 H=16 N=1024 d=64 fp32 causal (the fp32 tensor-core path)"),
     "causal_b1h32_n16384_d128": Workload(
         "causal_b1h32_n16384_d128", 1, 32, 16384, 16384, 128, 128, "bf16", True, 5,
         doc="long context B=1 H=32 N=16384 d=128 bf16 causal"),

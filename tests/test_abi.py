@@ -86,9 +86,14 @@ def test_argument_checks_backward(L):
 def test_tensor_path_request_rejects_other_shapes(L):
     try:
         L.attn_set_path(L.ATTN_PATH_TENSOR)
-        assert fwd(L, dt=0) == 4          # fp32 has no tensor-core path
-        assert fwd(L, d=32, dv=32) == 4
+        assert fwd(L, dt=0, d=72, dv=72) == 4     # fp32 on the tensor cores: widths <= 64
+        assert fwd(L, dt=0, d=62, dv=62) == 4     # ... and multiples of 4
+        assert fwd(L, dt=0, d=64, dv=96) == 4
+        assert fwd(L, d=32, dv=32) == 4           # bf16: d == dv in {64, 128}
         assert fwd(L, d=64, dv=128) == 4
+        if not torch.cuda.is_available():
+            assert fwd(L, dt=0, d=40, dv=24) == 7  # accepted; fails only at the launch
+            assert bwd(L, dt=0, d=64, dv=64) == 7
     finally:
         L.attn_set_path(L.ATTN_PATH_AUTO)
     assert L.lib.attn_set_path(9) == 4
