@@ -118,6 +118,61 @@ __device__ __forceinline__ void load_split(const float* __restrict__ src, int ro
     }
 }
 
+// Asynchronous 16-byte global -> shared copies (zero-filled past src_bytes).
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(sdst)),
+                 "l"(gsrc), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// The fp32 rows that load_split would read, copied as they are into `stage`
+// (32 bytes per 8-column chunk, in chunk order) without waiting. Each thread
+// copies the chunks it will later split itself (split_staged), so neither
+// step needs a barrier. The caller commits the copies as one group.
+template <int R, int NT>
+__device__ __forceinline__ void fetch(const float* __restrict__ src, int row0, int rows_valid,
+                                      int width, uint8_t* stage, int tid) {
+#pragma unroll 2
+    for (int k = tid; k < R * 8; k += NT) {
+        const int r = k >> 3, col = 8 * (k & 7);
+        const int grow = row0 + r;
+        const bool rv = grow < rows_valid;
+        const float* g = rv ? src + size_t(grow) * width + col : src;
+        const uint32_t n0 = (rv && col < width) ? 16u : 0u;
+        const uint32_t n1 = (rv && col + 4 < width) ? 16u : 0u;
+        cp_async16(stage + 32 * k, n0 ? g : src, n0);
+        cp_async16(stage + 32 * k + 16, n1 ? g + 4 : src, n1);
+    }
+}
+
+// Wait for this thread's copies, then split its chunks of `stage` into the
+// three pieces at `dst` (layout as load_split).
+template <int R, int NT>
+__device__ __forceinline__ void split_staged(const uint8_t* stage, uint8_t* dst, int tid) {
+    cp_async_wait_all();
+#pragma unroll 2
+    for (int k = tid; k < R * 8; k += NT) {
+        const int r = k >> 3, c = k & 7;
+        const float4 a = *reinterpret_cast<const float4*>(stage + 32 * k);
+        const float4 b = *reinterpret_cast<const float4*>(stage + 32 * k + 16);
+        uint4 p0, p1, p2;
+        split2(a.x, a.y, p0.x, p1.x, p2.x);
+        split2(a.z, a.w, p0.y, p1.y, p2.y);
+        split2(b.x, b.y, p0.z, p1.z, p2.z);
+        split2(b.z, b.w, p0.w, p1.w, p2.w);
+        const int off = r * 128 + ((c ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst + off) = p0;
+        *reinterpret_cast<uint4*>(dst + R * 128 + off) = p1;
+        *reinterpret_cast<uint4*>(dst + 2 * R * 128 + off) = p2;
+    }
+}
+
 // 32 values of this thread's row into the three pieces in TMEM: piece a of
 // the 64-wide row at columns col + 32 a .. +31 (two bf16 per column), this
 // half (h = 0, 1) at +16 h.
@@ -178,6 +233,7 @@ __device__ __forceinline__ void init_bars(Bars* bars, uint32_t tmem_cols) {
 // Wait until every MMA issued by thread 0 has completed, then free TMEM.
 __device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem, uint32_t tmem_cols,
                                          uint64_t budget_ns) {
+    cp_async_wait_all();
     if (threadIdx.x == 0) {
         mma_commit(&bars->drain);
         if (!mbar_wait_timed(&bars->drain, 0, budget_ns)) record_device_error(kErrTimeout);
@@ -220,7 +276,9 @@ constexpr uint32_t kFwdColS = 0, kFwdColPV = 64, kFwdColP = 128, kFwdTmemCols = 
 constexpr int kFwdOffQ = 0;
 constexpr int kFwdOffK = kFwdOffQ + kBigTile;          // two buffers
 constexpr int kFwdOffV = kFwdOffK + 2 * kSmallTile;    // two buffers
-constexpr int kFwdOffBar = kFwdOffV + 2 * kSmallTile;
+constexpr int kStageBytes = kSmall * 8 * 32;           // one fp32 64 x 64 tile in flight
+constexpr int kFwdOffStage = kFwdOffV + 2 * kSmallTile; // K, V of tile t + 2
+constexpr int kFwdOffBar = kFwdOffStage + 2 * kStageBytes;
 constexpr int kFwdSmemBytes = kFwdOffBar + 128;
 
 // Grid: one CTA per (128-query tile, head), heads fastest; causal grids start
@@ -243,9 +301,19 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     const int nkt = (m + kSmall - 1) / kSmall;
     const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
 
+    uint8_t* stK = smem + kFwdOffStage;
+    uint8_t* stV = stK + kStageBytes;
+    auto fetch_kv = [&](int t) {
+        fetch<kSmall, kThreads>(Kh, t * kSmall, m, d, stK, tid);
+        fetch<kSmall, kThreads>(Vh, t * kSmall, m, dv, stV, tid);
+        cp_async_commit();
+    };
+
     init_bars(bars, kFwdTmemCols);
     const bool aligned = (smem_addr(smem) & 1023u) == 0;
     if (aligned) {
+        // Key tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
+        if (T > 2) fetch_kv(2);
         load_split<kBig, kThreads>(Qh, q0, n, d, smem + kFwdOffQ, tid);
         load_split<kSmall, kThreads>(Kh, 0, m, d, smem + kFwdOffK, tid);
         load_split<kSmall, kThreads>(Vh, 0, m, dv, smem + kFwdOffV, tid);
@@ -335,11 +403,14 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
             tmem_row64(tl + kFwdColPV, pv);
 #pragma unroll
             for (int c = 0; c < 64; ++c) o[c] = fmaf(o[c], alpha, pv[c]);
-            // K_j (read by S_j) and V_j (read by P_j V_j) are free: tile j + 2.
+            // K_j (read by S_j) and V_j (read by P_j V_j) are free: split
+            // tile j + 2 from the staging buffer into them, then start
+            // fetching tile j + 3.
             if (j + 2 < T) {
-                load_split<kSmall, kThreads>(Kh, (j + 2) * kSmall, m, d, smem + kFwdOffK + buf * kSmallTile, tid);
-                load_split<kSmall, kThreads>(Vh, (j + 2) * kSmall, m, dv, smem + kFwdOffV + buf * kSmallTile, tid);
+                split_staged<kSmall, kThreads>(stK, smem + kFwdOffK + buf * kSmallTile, tid);
+                split_staged<kSmall, kThreads>(stV, smem + kFwdOffV + buf * kSmallTile, tid);
                 fence_proxy_async_smem();
+                if (j + 3 < T) fetch_kv(j + 3);
             }
         }
         tc_fence_before();
@@ -416,7 +487,8 @@ constexpr int kKvOffV = kKvOffK + kBigTile;
 constexpr int kKvOffQ = kKvOffV + kBigTile;            // two buffers
 constexpr int kKvOffdO = kKvOffQ + 2 * kSmallTile;     // two buffers
 constexpr int kKvOffRow = kKvOffdO + 2 * kSmallTile;   // [2][LSE 64 | D 64] floats
-constexpr int kKvOffBar = kKvOffRow + 4 * kSmall * 4;
+constexpr int kKvOffStage = kKvOffRow + 4 * kSmall * 4; // Q, dO, LSE | D of tile t + 2
+constexpr int kKvOffBar = kKvOffStage + 2 * kStageBytes + 2 * kSmall * 4;
 constexpr int kKvSmemBytes = kKvOffBar + 128;
 
 // Grid: one CTA per (128-key tile, head), heads fastest; causal grids start
@@ -445,18 +517,38 @@ bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
     const int i0 = causal ? k0 / kSmall : 0;
     const int T = nqs - i0;            // >= 1: causal has n == m > k0
 
+    // rows < n_pad: 64-row tiles never pass the 128-row padding
     auto load_q = [&](int idx, int buf) {
         const int r0 = (i0 + idx) * kSmall;
         load_split<kSmall, kBwdThreads>(Qh, r0, n, d, smem + kKvOffQ + buf * kSmallTile, tid);
         load_split<kSmall, kBwdThreads>(dOh, r0, n, dv, smem + kKvOffdO + buf * kSmallTile, tid);
-        // rows < n_pad: 64-row tiles never pass the 128-row padding
         if (tid < kSmall) sRow[buf * 128 + tid] = L2h[r0 + tid];
         else if (tid < 2 * kSmall) sRow[buf * 128 + tid] = Dh[r0 + tid - kSmall];
+    };
+    uint8_t* stQ = smem + kKvOffStage;
+    uint8_t* stdO = stQ + kStageBytes;
+    uint8_t* stRow = stdO + kStageBytes;                 // LSE 64 | D 64 floats
+    auto fetch_q = [&](int idx) {
+        const int r0 = (i0 + idx) * kSmall;
+        fetch<kSmall, kBwdThreads>(Qh, r0, n, d, stQ, tid);
+        fetch<kSmall, kBwdThreads>(dOh, r0, n, dv, stdO, tid);
+        if (tid < 16) cp_async16(stRow + 16 * tid, L2h + r0 + 4 * tid, 16);
+        else if (tid < 32) cp_async16(stRow + 16 * tid, Dh + r0 + 4 * (tid - 16), 16);
+        cp_async_commit();
+    };
+    auto split_q = [&](int buf) {
+        split_staged<kSmall, kBwdThreads>(stQ, smem + kKvOffQ + buf * kSmallTile, tid);
+        split_staged<kSmall, kBwdThreads>(stdO, smem + kKvOffdO + buf * kSmallTile, tid);
+        if (tid < 32)
+            *reinterpret_cast<float4*>(sRow + buf * 128 + 4 * tid) =
+                *reinterpret_cast<const float4*>(stRow + 16 * tid);
     };
 
     init_bars(bars, kKvTmemCols);
     const bool aligned = (smem_addr(smem) & 1023u) == 0;
     if (aligned) {
+        // Query tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
+        if (T > 2) fetch_q(2);
         load_split<kBig, kBwdThreads>(Kh, k0, m, d, smem + kKvOffK, tid);
         load_split<kBig, kBwdThreads>(Vh, k0, m, dv, smem + kKvOffV, tid);
         load_q(0, 0);
@@ -531,10 +623,12 @@ bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
             tc_fence_after();
             add_tmem32(tl + kKvColdV, acc_v);
             add_tmem32(tl + kKvColdK, acc_k);
-            // Q_i, dO_i, their LSE and D are free once dV, dK of this tile are done.
+            // Q_i, dO_i, their LSE and D are free once dV, dK of this tile
+            // are done: tile idx + 2 goes there, tile idx + 3 starts arriving.
             if (idx + 2 < T) {
-                load_q(idx + 2, buf);
+                split_q(buf);
                 fence_proxy_async_smem();
+                if (idx + 3 < T) fetch_q(idx + 3);
             }
         }
         tc_fence_before();
@@ -562,7 +656,8 @@ constexpr int kDqOffQ = 0;
 constexpr int kDqOffdO = kDqOffQ + kBigTile;
 constexpr int kDqOffK = kDqOffdO + kBigTile;           // two buffers
 constexpr int kDqOffV = kDqOffK + 2 * kSmallTile;      // two buffers
-constexpr int kDqOffBar = kDqOffV + 2 * kSmallTile;
+constexpr int kDqOffStage = kDqOffV + 2 * kSmallTile;  // K, V of tile t + 2
+constexpr int kDqOffBar = kDqOffStage + 2 * kStageBytes;
 constexpr int kDqSmemBytes = kDqOffBar + 128;
 
 // Grid as the forward's.
@@ -590,9 +685,19 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
     const int nkt = (m + kSmall - 1) / kSmall;
     const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
 
+    uint8_t* stK = smem + kDqOffStage;
+    uint8_t* stV = stK + kStageBytes;
+    auto fetch_kv = [&](int t) {
+        fetch<kSmall, kBwdThreads>(Kh, t * kSmall, m, d, stK, tid);
+        fetch<kSmall, kBwdThreads>(Vh, t * kSmall, m, dv, stV, tid);
+        cp_async_commit();
+    };
+
     init_bars(bars, kDqTmemCols);
     const bool aligned = (smem_addr(smem) & 1023u) == 0;
     if (aligned) {
+        // Key tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
+        if (T > 2) fetch_kv(2);
         load_split<kBig, kBwdThreads>(Qh, q0, n, d, smem + kDqOffQ, tid);
         load_split<kBig, kBwdThreads>(dOh, q0, n, dv, smem + kDqOffdO, tid);
         load_split<kSmall, kBwdThreads>(Kh, 0, m, d, smem + kDqOffK, tid);
@@ -665,13 +770,13 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
         if (got2) {
             tc_fence_after();
             add_tmem32(tl + kDqColdQ, acc);
-            // K_j (read by S_j and dS_j K_j) and V_j (read by dP_j) are free.
+            // K_j (read by S_j and dS_j K_j) and V_j (read by dP_j) are free:
+            // tile j + 2 goes there, tile j + 3 starts arriving.
             if (j + 2 < T) {
-                load_split<kSmall, kBwdThreads>(Kh, (j + 2) * kSmall, m, d,
-                                                smem + kDqOffK + buf * kSmallTile, tid);
-                load_split<kSmall, kBwdThreads>(Vh, (j + 2) * kSmall, m, dv,
-                                                smem + kDqOffV + buf * kSmallTile, tid);
+                split_staged<kSmall, kBwdThreads>(stK, smem + kDqOffK + buf * kSmallTile, tid);
+                split_staged<kSmall, kBwdThreads>(stV, smem + kDqOffV + buf * kSmallTile, tid);
                 fence_proxy_async_smem();
+                if (j + 3 < T) fetch_kv(j + 3);
             }
         }
         tc_fence_before();
