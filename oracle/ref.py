@@ -15,6 +15,11 @@ known mistake:
       S_ij = -inf for j > i             only if causal (then n == m)
       P = softmax(S) row by row         stable: subtract the row max
       O = P V
+  Optional padding mask ("Is there any Reference About Backpropagation of
+  the Transformer's Multi-Head Layer?", section 4, "Practical Tips for
+  Implementers": causal or padding masks go before the softmax, and the
+  backward then zeroes the masked gradients):
+      S_ij = -inf for j >= key_len[b]   keys past batch element b's length
   plus the per-row log-sum-exp LSE_i = log sum_j exp(S_ij). The pages do not
   define it. This oracle reads it as the natural log over the unmasked,
   already scaled scores, so that P = exp(S - LSE).
@@ -57,7 +62,9 @@ L = sum(O * dO); float64 torch autograd of the library's
 scaled_dot_product_attention; the explicit softmax Jacobian diag(a) - a a^T
 ("Lesson 4", Exercise 2); the rowsum(dP * P) = rowsum(dO * O) identity
 ("Attention Backpropagation: Step by step derivation", "Gradient of S");
-exact zeros at masked positions ("Attention backward", Problem 8); and
+exact zeros at masked positions ("Attention backward", Problem 8); the
+padding mask against the unmasked definition on keys cut to the valid
+length, and against finite differences; and
 mutation tests that plant each of the pages' wrong variants and check that
 the pins catch it. No function here is left unpinned.
 """
@@ -68,7 +75,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "default_scale", "scores", "apply_causal_mask", "row_softmax",
+    "default_scale", "scores", "apply_causal_mask", "apply_padding_mask", "row_softmax",
     "grad_v", "grad_p", "softmax_jvp", "grad_q", "grad_k",
     "head_forward", "head_backward",
     "attention_forward", "attention_backward",
@@ -102,6 +109,16 @@ def apply_causal_mask(S: np.ndarray, row0: int) -> np.ndarray:
     rows = np.arange(row0, row0 + S.shape[0])[:, None]
     cols = np.arange(S.shape[1])[None, :]
     return np.where(cols > rows, -np.inf, S)
+
+
+def apply_padding_mask(S: np.ndarray, key_len: int) -> np.ndarray:
+    """Set S_ij = -inf for every key j at or past ``key_len``, before the
+    softmax ("Is there any Reference ...", section 4: padding masks are
+    applied before the softmax). The pages name padding masks without a
+    layout; here they are given as the number of valid keys of each batch
+    element, the keys after it being padding."""
+    cols = np.arange(S.shape[1])[None, :]
+    return np.where(cols >= key_len, -np.inf, S)
 
 
 def row_softmax(S: np.ndarray):
@@ -158,32 +175,42 @@ def _check_head(Q, K, V, causal):
         raise ValueError("causal attention needs as many queries as keys")
 
 
-def _block_probs(Q, K, r0, r1, causal, scale):
+def _block_probs(Q, K, r0, r1, causal, scale, key_len=None):
     S = scores(Q[r0:r1], K, scale)
     if causal:
         S = apply_causal_mask(S, r0)
+    if key_len is not None:
+        S = apply_padding_mask(S, key_len)
     return row_softmax(S)
 
 
-def head_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK):
-    """Return (O, lse) for one head, in float64."""
+def _check_key_len(key_len, m):
+    if key_len is not None and not 1 <= key_len <= m:
+        raise ValueError(f"key_len {key_len} outside [1, {m}]")
+
+
+def head_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK, key_len=None):
+    """Return (O, lse) for one head, in float64. ``key_len``: number of
+    unpadded keys (None: all)."""
     Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
     _check_head(Q, K, V, causal)
+    _check_key_len(key_len, K.shape[0])
     scale = default_scale(Q.shape[1]) if scale is None else float(scale)
     n = Q.shape[0]
     O = np.empty((n, V.shape[1]))
     lse = np.empty(n)
     for r0 in range(0, n, row_block):
         r1 = min(n, r0 + row_block)
-        P, lse[r0:r1] = _block_probs(Q, K, r0, r1, causal, scale)
+        P, lse[r0:r1] = _block_probs(Q, K, r0, r1, causal, scale, key_len)
         O[r0:r1] = P @ V
     return O, lse
 
 
-def head_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
+def head_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK, key_len=None):
     """Return (dQ, dK, dV) for one head, in float64, recomputing P."""
     Q, K, V, dO = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, dO))
     _check_head(Q, K, V, causal)
+    _check_key_len(key_len, K.shape[0])
     scale = default_scale(Q.shape[1]) if scale is None else float(scale)
     n = Q.shape[0]
     dQ = np.empty_like(Q)
@@ -191,7 +218,7 @@ def head_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
     dV = np.zeros_like(V)
     for r0 in range(0, n, row_block):
         r1 = min(n, r0 + row_block)
-        P, _ = _block_probs(Q, K, r0, r1, causal, scale)
+        P, _ = _block_probs(Q, K, r0, r1, causal, scale, key_len)
         dV += grad_v(P, dO[r0:r1])
         dP = grad_p(dO[r0:r1], V)
         dS = softmax_jvp(P, dP)
@@ -210,17 +237,30 @@ def _heads(*arrays):
     return lead, flat
 
 
-def attention_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK):
-    """O and LSE for tensors shaped [..., n, d]; scale defaults to 1/sqrt(d)."""
+def _head_key_len(key_len, lead, h):
+    """The key length of flattened head h: key_len is indexed by the first
+    leading dimension (the batch) of [B, H, N, d] tensors."""
+    if key_len is None:
+        return None
+    per_batch = int(np.prod(lead[1:])) if len(lead) > 1 else 1
+    return int(key_len[h // per_batch])
+
+
+def attention_forward(Q, K, V, causal=False, scale=None, row_block=ROW_BLOCK, key_len=None):
+    """O and LSE for tensors shaped [..., n, d]; scale defaults to 1/sqrt(d).
+    ``key_len`` (optional, one entry per batch element): valid keys of each
+    batch element, the rest masked as padding."""
     lead, (q, k, v) = _heads(Q, K, V)
     O = np.empty(q.shape[:2] + (v.shape[2],))
     lse = np.empty(q.shape[:2])
     for h in range(q.shape[0]):
-        O[h], lse[h] = head_forward(q[h], k[h], v[h], causal, scale, row_block)
+        O[h], lse[h] = head_forward(q[h], k[h], v[h], causal, scale, row_block,
+                                    _head_key_len(key_len, lead, h))
     return O.reshape(lead + O.shape[1:]), lse.reshape(lead + lse.shape[1:])
 
 
-def attention_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK):
+def attention_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOCK,
+                       key_len=None):
     """(dQ, dK, dV) with the shapes of Q, K, V, for tensors shaped [..., N, d]."""
     lead, (q, k, v, do) = _heads(Q, K, V, dO)
     dQ = np.empty_like(q)
@@ -228,7 +268,8 @@ def attention_backward(Q, K, V, dO, causal=False, scale=None, row_block=ROW_BLOC
     dV = np.empty_like(v)
     for h in range(q.shape[0]):
         dQ[h], dK[h], dV[h] = head_backward(q[h], k[h], v[h], do[h], causal,
-                                            scale, row_block)
+                                            scale, row_block,
+                                            _head_key_len(key_len, lead, h))
     return (dQ.reshape(lead + dQ.shape[1:]), dK.reshape(lead + dK.shape[1:]),
             dV.reshape(lead + dV.shape[1:]))
 

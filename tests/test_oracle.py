@@ -416,7 +416,7 @@ def test_mask_after_softmax_is_caught(monkeypatch):
     """'Attention backward', wrong turn 5: zeroing A after the softmax."""
     assert _pins_pass()
 
-    def masked_late(Q, K, r0, r1, causal, scale):
+    def masked_late(Q, K, r0, r1, causal, scale, key_len=None):
         S = ref.scores(Q[r0:r1], K, scale)
         P, lse = ref.row_softmax(S)
         if causal:
@@ -599,3 +599,140 @@ def test_output_projection_backward_mutant_fails(monkeypatch):
                         lambda T, H: T.reshape(T.shape[0], T.shape[1], T.shape[2] // H, H).transpose(0, 3, 1, 2))
     bad, _ = ref.output_projection_backward(O, Wo, G)
     assert np.max(np.abs(bad - good)) > 1e-3
+
+
+# --------------------------------------------------------------------------
+# Padding mask ("Is there any Reference About Backpropagation of the
+# Transformer's Multi-Head Layer?", section 4: causal or padding masks go
+# before the softmax; the backward then zeroes the masked gradients). Keys at
+# or past key_len[b] of batch element b are padding.
+# --------------------------------------------------------------------------
+def _torch_padded(Q, K, V, dO, causal, scale, key_len):
+    """float64 torch autograd with an explicit boolean attention mask."""
+    B, H, n, _ = Q.shape
+    m = K.shape[2]
+    keep = torch.zeros(B, 1, n, m, dtype=torch.bool)
+    for b in range(B):
+        keep[b, :, :, :key_len[b]] = True
+    if causal:
+        keep &= ~torch.ones(n, m, dtype=torch.bool).triu(1)
+    q, k, v = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V))
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=keep, scale=scale)
+    o.backward(torch.tensor(dO, dtype=torch.float64))
+    sc = scale if scale is not None else 1 / math.sqrt(Q.shape[-1])
+    s = ((q @ k.transpose(-1, -2)) * sc).masked_fill(~keep, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return (o.detach().numpy(), lse.detach().numpy(), q.grad.numpy(), k.grad.numpy(),
+            v.grad.numpy())
+
+
+PADDED_CASES = [
+    # B, H, n, m, d, dv, causal, key_len, scale, seed
+    (2, 2, 7, 9, 4, 3, False, [4, 9], None, 0),
+    (3, 1, 8, 8, 5, 5, True, [3, 8, 1], None, 1),
+    (2, 3, 12, 12, 6, 4, True, [7, 12], 0.3, 2),
+    (1, 2, 5, 20, 8, 8, False, [13], None, 3),
+]
+
+
+def _padded_inputs(B, H, n, m, d, dv, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, n, d)), rng.standard_normal((B, H, m, d)),
+            rng.standard_normal((B, H, m, dv)), rng.standard_normal((B, H, n, dv)))
+
+
+def _padded_pins_pass():
+    try:
+        for (B, H, n, m, d, dv, causal, kl, scale, seed) in PADDED_CASES:
+            Q, K, V, dO = _padded_inputs(B, H, n, m, d, dv, seed)
+            got = ref.attention_forward(Q, K, V, causal, scale, row_block=3, key_len=kl) + \
+                ref.attention_backward(Q, K, V, dO, causal, scale, row_block=3, key_len=kl)
+            want = _torch_padded(Q, K, V, dO, causal, scale, kl)
+            if not all(rel_to_max(a, b) < 1e-12 for a, b in zip(got, want)):
+                return False
+    except Exception:
+        return False
+    return True
+
+
+def test_padding_mask_matches_torch_autograd_float64():
+    assert _padded_pins_pass()
+
+
+def test_padding_mask_equals_truncated_keys():
+    """Without the causal mask, padded keys behave as if they were absent:
+    O, LSE and dQ equal the unmasked attention on K[:L], V[:L]; dK and dV
+    match it on the first L rows and are exactly zero after them."""
+    Q, K, V, dO = _padded_inputs(2, 2, 6, 10, 4, 3, 7)
+    key_len = [3, 10]
+    O, lse = ref.attention_forward(Q, K, V, False, None, key_len=key_len)
+    dQ, dK, dV = ref.attention_backward(Q, K, V, dO, False, None, key_len=key_len)
+    for b, L in enumerate(key_len):
+        for h in range(2):
+            O_t, lse_t = ref.head_forward(Q[b, h], K[b, h, :L], V[b, h, :L])
+            dQ_t, dK_t, dV_t = ref.head_backward(Q[b, h], K[b, h, :L], V[b, h, :L], dO[b, h])
+            np.testing.assert_allclose(O[b, h], O_t, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lse[b, h], lse_t, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(dQ[b, h], dQ_t, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(dK[b, h, :L], dK_t, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(dV[b, h, :L], dV_t, rtol=0, atol=1e-13)
+            assert np.all(dK[b, h, L:] == 0.0) and np.all(dV[b, h, L:] == 0.0)
+
+
+def test_padding_mask_finite_differences():
+    rng = np.random.default_rng(21)
+    Q, K, V, dO = (rng.standard_normal(s) for s in ((5, 3), (6, 3), (6, 2), (5, 2)))
+    for causal, L in ((False, 4), (False, 1), (True, 4)):
+        if causal:
+            Qc, dOc = Q[:, :], dO[:, :]
+            Kc, Vc = K[:5], V[:5]
+        else:
+            Qc, dOc, Kc, Vc = Q, dO, K, V
+
+        def loss():
+            O, _ = ref.head_forward(Qc, Kc, Vc, causal, None, key_len=L)
+            return float(np.sum(O * dOc))
+
+        an = ref.head_backward(Qc, Kc, Vc, dOc, causal, None, key_len=L)
+        for p, a in zip((Qc, Kc, Vc), an):
+            num = np.zeros_like(p)
+            for idx in np.ndindex(p.shape):
+                orig = p[idx]
+                p[idx] = orig + 1e-5
+                lp = loss()
+                p[idx] = orig - 1e-5
+                lm = loss()
+                p[idx] = orig
+                num[idx] = (lp - lm) / 2e-5
+            assert max_rel_err(a, num) < 1e-6
+
+
+def test_padding_mask_after_softmax_is_caught(monkeypatch):
+    """Masking the padded weights after the softmax (the wrong turn the tip
+    warns about) leaves rows that do not sum to one: the pins fail."""
+    assert _padded_pins_pass()
+    orig = ref._block_probs
+
+    def masked_late(Q, K, r0, r1, causal, scale, key_len=None):
+        P, lse = orig(Q, K, r0, r1, causal, scale, None)
+        if key_len is not None:
+            P = P * (np.arange(P.shape[1])[None, :] < key_len)
+        return P, lse
+
+    monkeypatch.setattr(ref, "_block_probs", masked_late)
+    assert not _padded_pins_pass()
+
+
+def test_padding_mask_off_by_one_is_caught(monkeypatch):
+    assert _padded_pins_pass()
+    monkeypatch.setattr(ref, "apply_padding_mask",
+                        lambda S, L: np.where(np.arange(S.shape[1])[None, :] > L, -np.inf, S))
+    assert not _padded_pins_pass()
+
+
+def test_padding_key_len_out_of_range():
+    Q, K, V, dO = _padded_inputs(1, 1, 3, 4, 2, 2, 0)
+    with pytest.raises(ValueError):
+        ref.attention_forward(Q, K, V, key_len=[0])
+    with pytest.raises(ValueError):
+        ref.attention_backward(Q, K, V, dO, key_len=[5])
