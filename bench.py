@@ -113,8 +113,12 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def counted_bwd_flops_per_head(w: synth.Workload) -> float:
-    return w.bwd_flops() / (w.B * w.H)
+def metric_for(w: synth.Workload) -> str:
+    """The headline metric, with its precision and mask tags for the workload."""
+    tags = ["bf16" if w.dtype == "bf16" else "fp32", "causal" if w.causal else "non-causal"]
+    if w.key_len() is not None:
+        tags.append("key padding mask")
+    return METRIC.replace("(bf16, causal)", "(" + ", ".join(tags) + ")")
 
 
 class ClockSampler:
@@ -226,6 +230,8 @@ def run_ours(args, w, rank, world, local):
     lib.attn_set_path({"auto": lib.ATTN_PATH_AUTO, "simt": lib.ATTN_PATH_SIMT,
                        "tensor": lib.ATTN_PATH_TENSOR}[args.path])
     q, k, v, do = (t.to(dev) for t in synth.make_inputs(w, seed=w.seed + 1000 * rank))
+    kl_list = w.key_len()
+    kl = None if kl_list is None else torch.tensor(kl_list, dtype=torch.int32, device=dev)
     o = torch.empty((w.B, w.H, w.n, w.dv), dtype=q.dtype, device=dev)
     lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -241,11 +247,11 @@ def run_ours(args, w, rank, world, local):
             flush.zero_()
         if evs:
             evs[0].record()
-        lib.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        lib.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, key_len=kl)
         if evs:
             evs[1].record()
         lib.attn_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws,
-                     dq=dq, dk=dk, dv=dv)
+                     dq=dq, dk=dk, dv=dv, key_len=kl)
         if evs:
             evs[2].record()
 
@@ -307,15 +313,18 @@ def run_ours(args, w, rank, world, local):
     # step i's kernels, as a training loop feeding the library would.
     e2e = None
     if args.e2e_steps > 0:
-        pin_in = [[t.to("cpu").pin_memory() for t in (q, k, v, do)] for _ in range(2)]
+        ins = (q, k, v, do) if kl is None else (q, k, v, do, kl)
+        pin_in = [[t.to("cpu").pin_memory() for t in ins] for _ in range(2)]
         pin_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
                    for _ in range(2)]
         dev_sets = []
         for b in range(2):
+            kl_b = kl if (kl is None or b == 0) else torch.empty_like(kl)
             if b == 0:
-                dev_sets.append((q, k, v, do, o, lse, dq, dk, dv, ws))
+                dev_sets.append((q, k, v, do, o, lse, dq, dk, dv, ws, kl_b))
             else:
-                dev_sets.append(tuple(torch.empty_like(t) for t in (q, k, v, do, o, lse, dq, dk, dv, ws)))
+                dev_sets.append(tuple(torch.empty_like(t) for t in (q, k, v, do, o, lse, dq, dk, dv, ws))
+                                + (kl_b,))
         h2d = sum(t.numel() * t.element_size() for t in pin_in[0])
         d2h = sum(t.numel() * t.element_size() for t in pin_out[0])
         s_in, s_run, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
@@ -327,16 +336,18 @@ def run_ours(args, w, rank, world, local):
 
         def e2e_step(i):
             b = i % 2
-            qb, kb, vb, dob, ob, lseb, dqb, dkb, dvb, wsb = dev_sets[b]
+            qb, kb, vb, dob, ob, lseb, dqb, dkb, dvb, wsb, klb = dev_sets[b]
             s_in.wait_event(ev_free[b])
             with torch.cuda.stream(s_in):
-                for src, dst in zip(pin_in[b], (qb, kb, vb, dob)):
+                dsts = (qb, kb, vb, dob) if klb is None else (qb, kb, vb, dob, klb)
+                for src, dst in zip(pin_in[b], dsts):
                     dst.copy_(src, non_blocking=True)
                 ev_in[b].record(s_in)
             s_run.wait_event(ev_in[b])
-            lib.attn_fwd(qb, kb, vb, causal=w.causal, scale=w.scale, out=ob, lse=lseb, stream=s_run)
+            lib.attn_fwd(qb, kb, vb, causal=w.causal, scale=w.scale, out=ob, lse=lseb, stream=s_run,
+                         key_len=klb)
             lib.attn_bwd(qb, kb, vb, ob, dob, lseb, causal=w.causal, scale=w.scale, workspace=wsb,
-                         dq=dqb, dk=dkb, dv=dvb, stream=s_run)
+                         dq=dqb, dk=dkb, dv=dvb, stream=s_run, key_len=klb)
             ev_run[b].record(s_run)
             s_out.wait_event(ev_run[b])
             with torch.cuda.stream(s_out):
@@ -362,7 +373,7 @@ def run_ours(args, w, rank, world, local):
                "pipelined": "2 buffer sets, upload/compute/download streams"}
 
     result = {
-        "metric": METRIC if w.dtype == "bf16" else METRIC.replace("(bf16, causal)", f"(fp32, {'causal' if w.causal else 'non-causal'})"),
+        "metric": metric_for(w),
         "value": round(value, 3),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -377,6 +388,7 @@ def run_ours(args, w, rank, world, local):
         "config": {
             "workload": w.name, "B": w.B, "H": w.H, "n": w.n, "m": w.m, "d": w.d, "dv": w.dv,
             "causal": w.causal, "scale": w.scale, "path": args.path,
+            **({} if kl_list is None else {"key_len": kl_list}),
             "parallelism": "replicas" if world == 1 else f"independent (batch, head) problems x{world}",
             "l2": ("flushed between steps (256 MiB write)" if flush is not None else
                    f"inputs larger than L2 ({working_set / 2**20:.0f} MiB per step)"),
@@ -517,17 +529,20 @@ def oracle_sample(w, seconds, max_heads=None):
     have passed. Returns (TFLOP/s in the metric's counting, heads, elapsed)."""
     import oracle.ref as ref
     q, k, v, do = synth.make_inputs(w)
+    kl = w.key_len()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
-    done, t0 = 0, time.perf_counter()
+    done, flops, t0 = 0, 0.0, time.perf_counter()
     while True:
         b, h = heads[done % len(heads)]
         Q, K, V, dO = (t[b, h].to(torch.float64).numpy() for t in (q, k, v, do))
-        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale)
+        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale,
+                          key_len=None if kl is None else kl[b])
         done += 1
+        flops += w.head_bwd_flops(b)
         elapsed = time.perf_counter() - t0
         if elapsed >= seconds or (max_heads and done >= max_heads):
             break
-    return done * counted_bwd_flops_per_head(w) / elapsed / 1e12, done, elapsed
+    return flops / elapsed / 1e12, done, elapsed
 
 
 def run_reference(args, w, rank, world):
@@ -535,26 +550,28 @@ def run_reference(args, w, rank, world):
         return None
     import oracle.ref as ref
     q, k, v, do = synth.make_inputs(w)
+    kl = w.key_len()
     heads = [(b, h) for b in range(w.B) for h in range(w.H)]
 
     def one(i):
         b, h = heads[i % len(heads)]
         Q, K, V, dO = (t[b, h].to(torch.float64).numpy() for t in (q, k, v, do))
-        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale)
+        ref.head_backward(Q, K, V, dO, causal=w.causal, scale=w.scale,
+                          key_len=None if kl is None else kl[b])
+        return w.head_bwd_flops(b)
 
     for i in range(args.warmup):
         one(i)
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        one(i)
+    flops = sum(one(i) for i in range(args.steps))
     elapsed = time.perf_counter() - t0
-    value = args.steps * counted_bwd_flops_per_head(w) / elapsed / 1e12
+    value = flops / elapsed / 1e12
     cores = blas_threads()
     sample = (f"one (batch, head) problem of {w.name} per step "
               f"(n={w.n}, m={w.m}, d={w.d}), float64 oracle backward")
     return {
         "impl": "reference",
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "metric": metric_for(w), "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * elapsed / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

@@ -113,6 +113,38 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V,
                        attn_dtype_t dtype, int causal, float scale, void* stream);
 
 /*
+ * attn_fwd_masked, attn_bwd_masked -- attn_fwd and attn_bwd with a key
+ * padding mask ("Is there any Reference About Backpropagation of the
+ * Transformer's Multi-Head Layer?", section 4, "Practical Tips for
+ * Implementers": causal or padding masks go before the softmax, and the
+ * backward pass then zeroes the masked gradients). The pages give padding
+ * masks no layout; here the mask is
+ *   key_len  [B] int32 in device memory (4-byte aligned; NULL: no mask):
+ *            the number of valid keys of batch element b. Keys j >= key_len[b]
+ *            of every head of b get S = -inf before the softmax, so P = 0 and
+ *            dS = 0 there, and their dK and dV rows are zero. Values are
+ *            clamped to [1, m] on the device (a row with no valid key has no
+ *            softmax). Query rows are never masked: rows of padded queries
+ *            attend to the valid keys as usual.
+ * Both calls must see the same key_len; with causal != 0 the two masks
+ * combine. All other arguments, limits and errors are those of attn_fwd and
+ * attn_bwd, which are these calls with key_len = NULL. Key tiles made only of
+ * padding are skipped by the forward and do one masked query tile's work in
+ * the backward.
+ */
+attn_status_t attn_fwd_masked(const void* Q, const void* K, const void* V,
+                              void* O, float* LSE, const int* key_len,
+                              int B, int H, int n, int m, int d, int dv,
+                              attn_dtype_t dtype, int causal, float scale, void* stream);
+
+attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V,
+                              const void* O, const void* dO, const float* LSE,
+                              const int* key_len, void* dQ, void* dK, void* dV,
+                              void* workspace, size_t workspace_bytes,
+                              int B, int H, int n, int m, int d, int dv,
+                              attn_dtype_t dtype, int causal, float scale, void* stream);
+
+/*
  * attn_bwd_noalloc -- attn_bwd for callers that cannot allocate device memory.
  * The pages have no counterpart: this is a deployment convenience, not part
  * of the method. Some callers cannot hand attn_bwd a workspace: a plugin or

@@ -69,6 +69,11 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                            i, i, i, i, i, i, i, i, f, vp]
     L.attn_bwd.restype = i
+    L.attn_fwd_masked.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp]
+    L.attn_fwd_masked.restype = i
+    L.attn_bwd_masked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                  i, i, i, i, i, i, i, i, f, vp]
+    L.attn_bwd_masked.restype = i
     L.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i, i]
     L.attn_bwd_workspace_size.restype = sz
     L.attn_get_device_error.argtypes = [vp]
@@ -156,26 +161,47 @@ def attn_bwd_workspace_size(B, H, n, m, d, dv, dtype) -> int:
     return int(lib.attn_bwd_workspace_size(B, H, n, m, d, dv, code))
 
 
-def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
-    """Returns (O, LSE) for [B,H,N,d] CUDA tensors."""
+def _key_len(key_len, B, device):
+    """The padding mask argument: None, or an int32 [B] tensor on the device."""
+    if key_len is None:
+        return None
+    if (not isinstance(key_len, torch.Tensor) or key_len.dtype != torch.int32 or
+            key_len.shape != (B,) or key_len.device != device or not key_len.is_contiguous()):
+        raise ValueError("key_len must be a contiguous int32 [B] tensor on the inputs' device")
+    return key_len
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None, key_len=None):
+    """Returns (O, LSE) for [B,H,N,d] CUDA tensors. key_len (optional int32
+    [B] device tensor): valid keys per batch element; later keys are padding,
+    masked before the softmax (attn_fwd_masked)."""
     _require(q, k, v)
     B, H, n, m, d, dv = _dims(q, k, v)
+    key_len = _key_len(key_len, B, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty((B, H, n, dv), dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
-    _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, m, d, dv,
-                        dtype_code(q.dtype), int(bool(causal)), scale, _stream_handle(stream)),
-           "attn_fwd")
+    if key_len is None:
+        _check(lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, n, m, d, dv,
+                            dtype_code(q.dtype), int(bool(causal)), scale,
+                            _stream_handle(stream)), "attn_fwd")
+    else:
+        _check(lib.attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                   _ptr(key_len), B, H, n, m, d, dv, dtype_code(q.dtype),
+                                   int(bool(causal)), scale, _stream_handle(stream)),
+               "attn_fwd_masked")
     return out, lse
 
 
 def attn_bwd(q, k, v, o, do, lse, causal=False, scale=None, workspace=None,
-             dq=None, dk=None, dv=None, stream=None):
-    """Returns (dQ, dK, dV) with the shapes of Q, K, V."""
+             dq=None, dk=None, dv=None, stream=None, key_len=None):
+    """Returns (dQ, dK, dV) with the shapes of Q, K, V. key_len: the padding
+    mask given to attn_fwd (attn_bwd_masked)."""
     _require(q, k, v, o, do)
     B, H, n, m, d, dvw = _dims(q, k, v)
+    key_len = _key_len(key_len, B, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     code = dtype_code(q.dtype)
     need = attn_bwd_workspace_size(B, H, n, m, d, dvw, code)
@@ -187,12 +213,18 @@ def attn_bwd(q, k, v, o, do, lse, causal=False, scale=None, workspace=None,
         dk = torch.empty_like(k)
     if dv is None:
         dv = torch.empty_like(v)
-    _check(lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
-                        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-                        workspace.numel() * workspace.element_size(),
-                        B, H, n, m, d, dvw, code, int(bool(causal)), scale,
-                        _stream_handle(stream)),
-           "attn_bwd")
+    if key_len is None:
+        _check(lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                            _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(),
+                            B, H, n, m, d, dvw, code, int(bool(causal)), scale,
+                            _stream_handle(stream)), "attn_bwd")
+    else:
+        _check(lib.attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse),
+                                   _ptr(key_len), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(),
+                                   B, H, n, m, d, dvw, code, int(bool(causal)), scale,
+                                   _stream_handle(stream)), "attn_bwd_masked")
     return dq, dk, dv
 
 

@@ -70,6 +70,14 @@ attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, Path* path) {
     return ATTN_OK;
 }
 
+// The key padding mask as the kernels take it: valid keys per batch element
+// (device int32 [B], or null for none) and the head count that maps a
+// (batch, head) index to its batch element.
+struct Mask {
+    const int* key_len;
+    int H;
+};
+
 struct Workspace {
     size_t lse2_off, dd_off, dq_off, sched_off, total;
     int n_pad;
@@ -212,7 +220,8 @@ int grid_for(size_t work_items, int per_block, int cap) {
 
 template <typename T>
 attn_status_t fwd_simt(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH,
-                       int n, int m, int d, int dv, int causal, float scale, cudaStream_t st) {
+                       int n, int m, int d, int dv, int causal, float scale, Mask mask,
+                       cudaStream_t st) {
     const size_t smem = attn::simt::fwd_smem_bytes<T>(d, dv);
     auto kern = attn::simt::fwd_kernel<T>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -222,14 +231,15 @@ attn_status_t fwd_simt(const void* Q, const void* K, const void* V, void* O, flo
     return traced(ATTN_KERNEL_FWD_SIMT, st, [&] {
         kern<<<grid, attn::simt::kThreads, smem, st>>>(
             static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
-            static_cast<T*>(O), LSE, n, m, d, dv, causal, scale);
+            static_cast<T*>(O), LSE, n, m, d, dv, causal, scale, mask.key_len, mask.H);
         return launched();
     });
 }
 
 template <int D>
 attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, float* LSE,
-                         int BH, int n, int m, int causal, float scale, cudaStream_t st) {
+                         int BH, int n, int m, int causal, float scale, Mask mask,
+                         cudaStream_t st) {
     using C = attn::fwdtc::Cfg<D>;
     CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) || !make_map(&mv, V, D, m, BH) ||
@@ -247,7 +257,8 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
     const int head_group = std::max(1, std::min(BH, 256 / num_pairs));
     return traced(ATTN_KERNEL_FWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mo, LSE, n, m, BH, head_group, causal, scale * kLog2e, kWaitBudgetNs);
+            mq, mk, mv, mo, LSE, n, m, BH, head_group, causal, scale * kLog2e, mask.key_len,
+            mask.H, kWaitBudgetNs);
         return launched();
     });
 }
@@ -294,7 +305,7 @@ template <typename T>
 attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* dO,
                        const float* LSE, const float* Dd, int n_pad, float* dQacc, void* dK,
                        void* dV, int BH, int n, int m, int d, int dv, int causal, float scale,
-                       cudaStream_t st) {
+                       Mask mask, cudaStream_t st) {
     const size_t smem = attn::simt::bwd_smem_bytes<T>(d, dv);
     auto kern = attn::simt::bwd_kernel<T>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -305,7 +316,7 @@ attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* 
         kern<<<grid, attn::simt::kThreads, smem, st>>>(
             static_cast<const T*>(Q), static_cast<const T*>(K), static_cast<const T*>(V),
             static_cast<const T*>(dO), LSE, Dd, n_pad, dQacc, static_cast<T*>(dK),
-            static_cast<T*>(dV), n, m, d, dv, causal, scale);
+            static_cast<T*>(dV), n, m, d, dv, causal, scale, mask.key_len, mask.H);
         return launched();
     });
 }
@@ -313,7 +324,7 @@ attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* 
 template <int D>
 attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void* dO,
                          const float* lse2, const float* Dd, int* sched, int n_pad, float* dQacc, void* dK,
-                         void* dV, int BH, int n, int m, int causal, float scale,
+                         void* dV, int BH, int n, int m, int causal, float scale, Mask mask,
                          cudaStream_t st) {
     using C = attn::bwdtc::Cfg<D>;
     CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
@@ -337,7 +348,7 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
             mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, sched, n_pad, n, m, BH, head_group, causal, scale,
-            scale * kLog2e, kWaitBudgetNs);
+            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
         return launched();
     });
 }
@@ -351,7 +362,8 @@ attn_status_t f32x_grid(int rows, int BH, unsigned* grid) {
 }
 
 attn_status_t fwd_f32x(const void* Q, const void* K, const void* V, void* O, float* LSE, int BH,
-                       int n, int m, int d, int dv, int causal, float scale, cudaStream_t st) {
+                       int n, int m, int d, int dv, int causal, float scale, Mask mask,
+                       cudaStream_t st) {
     namespace fx = attn::f32x;
     unsigned grid = 0;
     attn_status_t s = f32x_grid(n, BH, &grid);
@@ -363,14 +375,14 @@ attn_status_t fwd_f32x(const void* Q, const void* K, const void* V, void* O, flo
         fx::fwd_kernel<<<grid, fx::kThreads, fx::kFwdSmemBytes, st>>>(
             static_cast<const float*>(Q), static_cast<const float*>(K),
             static_cast<const float*>(V), static_cast<float*>(O), LSE, n, m, d, dv, BH, causal,
-            scale * kLog2e, kWaitBudgetNs);
+            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
         return launched();
     });
 }
 
 attn_status_t bwd_f32x(const void* Q, const void* K, const void* V, const void* dO,
                        const float* lse2, const float* Dd, int n_pad, void* dQ, void* dK, void* dV,
-                       int BH, int n, int m, int d, int dv, int causal, float scale,
+                       int BH, int n, int m, int d, int dv, int causal, float scale, Mask mask,
                        cudaStream_t st) {
     namespace fx = attn::f32x;
     unsigned grid_kv = 0, grid_dq = 0;
@@ -389,14 +401,14 @@ attn_status_t bwd_f32x(const void* Q, const void* K, const void* V, const void* 
     s = traced(ATTN_KERNEL_BWD_F32X_KV, st, [&] {
         fx::bwd_kv_kernel<<<grid_kv, fx::kBwdThreads, fx::kKvSmemBytes, st>>>(
             q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dK), static_cast<float*>(dV), n, m,
-            d, dv, BH, causal, scale, scale * kLog2e, kWaitBudgetNs);
+            d, dv, BH, causal, scale, scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
         return launched();
     });
     if (s != ATTN_OK) return s;
     return traced(ATTN_KERNEL_BWD_F32X_DQ, st, [&] {
         fx::bwd_dq_kernel<<<grid_dq, fx::kBwdThreads, fx::kDqSmemBytes, st>>>(
             q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dQ), n, m, d, dv, BH, causal, scale,
-            scale * kLog2e, kWaitBudgetNs);
+            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
         return launched();
     });
 }
@@ -479,42 +491,53 @@ size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv, attn_d
     return carve(B, H, n, d).total;
 }
 
-attn_status_t attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                       int H, int n, int m, int d, int dv, attn_dtype_t dtype, int causal,
-                       float scale, void* stream) {
+attn_status_t attn_fwd_masked(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                              const int* key_len, int B, int H, int n, int m, int d, int dv,
+                              attn_dtype_t dtype, int causal, float scale, void* stream) {
     attn_status_t s = check_sizes(B, H, n, m, d, dv, dtype, causal);
     if (s != ATTN_OK) return s;
     if (!std::isfinite(scale)) return ATTN_ERR_SHAPE;
     if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_NULL;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+        (reinterpret_cast<uintptr_t>(key_len) & 3u) != 0)
         return ATTN_ERR_ALIGN;
     Path path = Path::kSimt;
     if ((s = choose_path(dtype, d, dv, &path)) != ATTN_OK) return s;
     const int BH = B * H;
+    const Mask mask{key_len, H};
     cudaStream_t st = as_stream(stream);
     if (path == Path::kTensorF32x)
-        s = fwd_f32x(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+        s = fwd_f32x(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, mask, st);
     else if (path == Path::kTensorBf16)
-        s = (d == 64) ? fwd_tensor<64>(Q, K, V, O, LSE, BH, n, m, causal, scale, st)
-                      : fwd_tensor<128>(Q, K, V, O, LSE, BH, n, m, causal, scale, st);
+        s = (d == 64) ? fwd_tensor<64>(Q, K, V, O, LSE, BH, n, m, causal, scale, mask, st)
+                      : fwd_tensor<128>(Q, K, V, O, LSE, BH, n, m, causal, scale, mask, st);
     else if (dtype == ATTN_F32)
-        s = fwd_simt<float>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+        s = fwd_simt<float>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, mask, st);
     else
-        s = fwd_simt<__nv_bfloat16>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, st);
+        s = fwd_simt<__nv_bfloat16>(Q, K, V, O, LSE, BH, n, m, d, dv, causal, scale, mask, st);
     if (s == ATTN_OK) g_last_launches = 1;
     return s;
 }
 
-attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* O,
-                       const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
-                       void* workspace, size_t workspace_bytes, int B, int H, int n, int m, int d,
-                       int dv, attn_dtype_t dtype, int causal, float scale, void* stream) {
+attn_status_t attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                       int H, int n, int m, int d, int dv, attn_dtype_t dtype, int causal,
+                       float scale, void* stream) {
+    return attn_fwd_masked(Q, K, V, O, LSE, nullptr, B, H, n, m, d, dv, dtype, causal, scale,
+                           stream);
+}
+
+attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, const int* key_len, void* dQ,
+                              void* dK, void* dV, void* workspace, size_t workspace_bytes, int B,
+                              int H, int n, int m, int d, int dv, attn_dtype_t dtype, int causal,
+                              float scale, void* stream) {
     attn_status_t s = check_sizes(B, H, n, m, d, dv, dtype, causal);
     if (s != ATTN_OK) return s;
     if (!std::isfinite(scale)) return ATTN_ERR_SHAPE;
     if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV) return ATTN_ERR_NULL;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) ||
-        !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+        !aligned16(LSE) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+        (reinterpret_cast<uintptr_t>(key_len) & 3u) != 0)
         return ATTN_ERR_ALIGN;
     const Workspace w = carve(B, H, n, d);
     if (!workspace || workspace_bytes < w.total) return ATTN_ERR_WORKSPACE;
@@ -524,6 +547,7 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     const bool tensor = path != Path::kSimt;
 
     const int BH = B * H;
+    const Mask mask{key_len, H};
     cudaStream_t st = as_stream(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
@@ -544,24 +568,32 @@ attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* 
     if (s != ATTN_OK) return s;
     if (path == Path::kTensorF32x) {
         s = bwd_f32x(Q, K, V, dO, lse2, Dd, w.n_pad, dQ, dK, dV, BH, n, m, d, dv, causal, scale,
-                     st);
+                     mask, st);
     } else if (path == Path::kTensorBf16) {
         s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
-                                       n, m, causal, scale, st)
+                                       n, m, causal, scale, mask, st)
                       : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
-                                        n, m, causal, scale, st);
+                                        n, m, causal, scale, mask, st);
         if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, 1.0f, st);
     } else if (dtype == ATTN_F32) {
         s = bwd_simt<float>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv, causal,
-                            scale, st);
+                            scale, mask, st);
         if (s == ATTN_OK) s = finalize<float>(dQacc, dQ, dq_elems, scale, st);
     } else {
         s = bwd_simt<__nv_bfloat16>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv,
-                                    causal, scale, st);
+                                    causal, scale, mask, st);
         if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, scale, st);
     }
     if (s == ATTN_OK) g_last_launches = 3;
     return s;
+}
+
+attn_status_t attn_bwd(const void* Q, const void* K, const void* V, const void* O,
+                       const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                       void* workspace, size_t workspace_bytes, int B, int H, int n, int m, int d,
+                       int dv, attn_dtype_t dtype, int causal, float scale, void* stream) {
+    return attn_bwd_masked(Q, K, V, O, dO, LSE, nullptr, dQ, dK, dV, workspace, workspace_bytes, B,
+                           H, n, m, d, dv, dtype, causal, scale, stream);
 }
 
 attn_status_t attn_trace_begin(int capacity) {

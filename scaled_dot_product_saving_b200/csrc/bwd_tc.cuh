@@ -54,6 +54,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "padmask.cuh"
 
 namespace attn {
 namespace bwdtc {
@@ -178,16 +179,21 @@ __device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int&
 }
 
 // One work item: 128 keys of one head and the query tiles that see them.
+// mk: the head's valid keys (the padding mask, or m). An item whose keys are
+// all padding visits one query tile, where every P is 0, so that its dK and
+// dV rows are still written (as zeros).
 struct Item {
-    int bh, k0, first_qt, T;
+    int bh, k0, first_qt, T, mk;
 };
-__device__ __forceinline__ Item item_at(int b, int num_kt, int num_qt, int BH, int hg, int causal) {
+__device__ __forceinline__ Item item_at(int b, int num_kt, int num_qt, int BH, int hg, int causal,
+                                        const int* key_len, int H, int m) {
     Item it;
     int kt;
     cta_tile(b, num_kt, BH, hg, it.bh, kt);
     it.k0 = kt * kBN;
+    it.mk = keys_valid(key_len, it.bh, H, m);
     it.first_qt = causal ? kt : 0;
-    it.T = num_qt - it.first_qt;          // >= 1
+    it.T = (it.k0 >= it.mk) ? 1 : num_qt - it.first_qt;          // >= 1
     return it;
 }
 
@@ -199,7 +205,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
            const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ lse2,
            const float* __restrict__ Dd, int* __restrict__ sched, int n_pad, int n, int m, int BH,
            int head_group, int causal, float scale, float scale_log2,
-           unsigned long long budget_ns) {
+           const int* __restrict__ key_len, int H, unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
@@ -219,7 +225,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     const int num_qt = (n + kBM - 1) / kBM;
     const int num_items = num_kt * BH;
     const int G = int(gridDim.x);
-    auto item = [&](int b) { return item_at(b, num_kt, num_qt, BH, head_group, causal); };
+    auto item = [&](int b) {
+        return item_at(b, num_kt, num_qt, BH, head_group, causal, key_len, H, m);
+    };
     // Consumers: the work item of the j-th slot (-1 = no more), or -2 if
     // the wait gave up. A warp reads it in every lane, then lane 0 releases
     // the slot; the MMA thread passes warp = false.
@@ -513,7 +521,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const Item it = item(b);
-            const bool key_ok = it.k0 + r < m;
+            const bool key_ok = it.k0 + r < it.mk;
             for (int t = 0; t < it.T; ++t, ++g) {
                 const int s = g % C::kStages;
                 const int q0 = (it.first_qt + t) * kBM;

@@ -45,6 +45,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "padmask.cuh"
 
 namespace attn {
 namespace f32x {
@@ -286,7 +287,8 @@ constexpr int kFwdSmemBytes = kFwdOffBar + 128;
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
            float* __restrict__ O, float* __restrict__ LSE, int n, int m, int d, int dv, int BH,
-           int causal, float scale_log2, unsigned long long budget_ns) {
+           int causal, float scale_log2, const int* __restrict__ key_len, int H,
+           unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kFwdOffBar);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -298,7 +300,8 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     const float* Qh = Q + size_t(bh) * n * d;
     const float* Kh = K + size_t(bh) * m * d;
     const float* Vh = V + size_t(bh) * m * dv;
-    const int nkt = (m + kSmall - 1) / kSmall;
+    const int mk = keys_valid(key_len, bh, H, m);        // keys past mk: padding
+    const int nkt = (mk + kSmall - 1) / kSmall;
     const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
 
     uint8_t* stK = smem + kFwdOffStage;
@@ -357,7 +360,7 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
             for (int c = 0; c < 64; ++c) {
                 const int key = kb + c;
                 float x = s[c] * scale_log2;
-                if (key >= m || (causal && key > row)) x = -INFINITY;
+                if (key >= mk || (causal && key > row)) x = -INFINITY;
                 s[c] = x;
                 mx = fmaxf(mx, x);
             }
@@ -498,7 +501,8 @@ bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
               const float* __restrict__ dO, const float* __restrict__ lse2,
               const float* __restrict__ Dd, int n_pad, float* __restrict__ dK,
               float* __restrict__ dV, int n, int m, int d, int dv, int BH, int causal, float scale,
-              float scale_log2, unsigned long long budget_ns) {
+              float scale_log2, const int* __restrict__ key_len, int H,
+              unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kKvOffBar);
     float* sRow = reinterpret_cast<float*>(smem + kKvOffRow);
@@ -515,7 +519,11 @@ bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
     const float* Dh = Dd + size_t(bh) * n_pad;
     const int nqs = (n + kSmall - 1) / kSmall;
     const int i0 = causal ? k0 / kSmall : 0;
-    const int T = nqs - i0;            // >= 1: causal has n == m > k0
+    // Keys past mk are padding: their rows get P = 0 and zero dK, dV; a tile
+    // of only padded keys visits one query tile so that the zeros are written.
+    const int mk = keys_valid(key_len, bh, H, m);
+    const bool key_dead = krow >= mk;
+    const int T = (k0 >= mk) ? 1 : nqs - i0;   // >= 1: causal has n == m > k0
 
     // rows < n_pad: 64-row tiles never pass the 128-row padding
     auto load_q = [&](int idx, int buf) {
@@ -591,7 +599,7 @@ bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
                 float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -Lrow[c]));
-                if (causal && krow > qb + c) pv = 0.f;
+                if (key_dead || (causal && krow > qb + c)) pv = 0.f;
                 sr[c] = __float_as_uint(pv);
                 pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -Drow[c]));
             }
@@ -666,7 +674,7 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
               const float* __restrict__ dO, const float* __restrict__ lse2,
               const float* __restrict__ Dd, int n_pad, float* __restrict__ dQ, int n, int m, int d,
               int dv, int BH, int causal, float scale, float scale_log2,
-              unsigned long long budget_ns) {
+              const int* __restrict__ key_len, int H, unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kDqOffBar);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -682,7 +690,8 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
     const float* dOh = dO + size_t(bh) * n * dv;
     const float l2 = lse2[size_t(bh) * n_pad + row];     // row < n_pad
     const float dd = Dd[size_t(bh) * n_pad + row];
-    const int nkt = (m + kSmall - 1) / kSmall;
+    const int mk = keys_valid(key_len, bh, H, m);        // keys past mk: padding
+    const int nkt = (mk + kSmall - 1) / kSmall;
     const int T = causal ? min(nkt, (q0 + kBig - 1) / kSmall + 1) : nkt;
 
     uint8_t* stK = smem + kDqOffStage;
@@ -743,7 +752,7 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
             for (int c = 0; c < 32; ++c) {
                 const int key = kb + c;
                 float pv = ex2(fmaf(__uint_as_float(sr[c]), scale_log2, -l2));
-                if (key >= m || (causal && key > row)) pv = 0.f;
+                if (key >= mk || (causal && key > row)) pv = 0.f;
                 pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -dd));
             }
             split32_to_tmem(pr, tl - 32 * half + kDqColdS + 16 * half);

@@ -47,6 +47,7 @@
 #pragma once
 
 #include "sm100.cuh"
+#include "padmask.cuh"
 
 namespace attn {
 namespace fwdtc {
@@ -153,15 +154,20 @@ __device__ __forceinline__ void chunk_p(const uint32_t (&r)[32], f32x2 sl2, f32x
 
 // One work item: the query-tile pair `pair` (tiles A = 2 pair, B = 2 pair + 1)
 // of one head, and the key tiles each tile needs.
+// mk: the head's valid keys (the padding mask, or m); key tiles past it are
+// not visited.
 struct Item {
-    int bh, qt[2], nkv[2], num_kv;
+    int bh, qt[2], nkv[2], num_kv, mk;
     bool has_b;
 };
-__device__ __forceinline__ Item item_at(int b, int num_qt, int num_kt, int BH, int hg, int causal) {
+__device__ __forceinline__ Item item_at(int b, int num_qt, int BH, int hg, int causal,
+                                        const int* key_len, int H, int m) {
     Item it;
     const int num_pairs = (num_qt + 1) / 2;
     int pair;
     cta_pair(b, num_pairs, BH, hg, it.bh, pair);
+    it.mk = keys_valid(key_len, it.bh, H, m);
+    const int num_kt = (it.mk + kBN - 1) / kBN;
     it.has_b = 2 * pair + 1 < num_qt;
     it.qt[0] = 2 * pair;
     it.qt[1] = 2 * pair + 1;
@@ -176,7 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
            float* __restrict__ LSE, int n, int m, int BH, int head_group, int causal,
-           float scale_log2, unsigned long long budget_ns) {
+           float scale_log2, const int* __restrict__ key_len, int H,
+           unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
@@ -184,8 +191,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_qt = (n + kBM - 1) / kBM;
-    const int num_kt = (m + kBN - 1) / kBN;
-    auto item = [&](int b) { return item_at(b, num_qt, num_kt, BH, head_group, causal); };
+    auto item = [&](int b) { return item_at(b, num_qt, BH, head_group, causal, key_len, H, m); };
     // Persistent through cluster launch control: a CTA starts with the work
     // item of its own index and, while it works, asks the hardware to cancel
     // the launch of a CTA that has not started and takes over that CTA's item
@@ -476,8 +482,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int q0 = (x ? it.qt[1] : it.qt[0]) * kBM;
             const int row = q0 + r;
             const int ntile = x ? it.nkv[1] : it.nkv[0];
-            // Keys after kmax are masked: past the end, or after the row (causal).
-            const int kmax = causal ? min(row, m - 1) : m - 1;
+            // Keys after kmax are masked: past the end or the padding mask,
+            // or after the row (causal).
+            const int kmax = causal ? min(row, it.mk - 1) : it.mk - 1;
             float m_run = -INFINITY, l_run = 0.f;
             for (int t = 0; t < ntile; ++t) {
                 if (!mbar_wait_warp(&bars->s_full[x], cx & 1, abort_flag, budget_ns)) {

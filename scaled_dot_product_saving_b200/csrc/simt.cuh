@@ -9,6 +9,8 @@
 // registers and adds dQ's share into an fp32 accumulator with atomics.
 #pragma once
 
+#include "padmask.cuh"
+
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -48,7 +50,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 fwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict__ V,
            T* __restrict__ O, float* __restrict__ LSE, int n, int m, int d, int dv,
-           int causal, float scale) {
+           int causal, float scale, const int* __restrict__ key_len, int H) {
     extern __shared__ float sm[];
     const int pk = odd_pitch(d);
     float* Qs = sm;                      // [64][d]
@@ -76,7 +78,8 @@ fwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict
         for (int k = 0; k < kCols; ++k) acc[rr][k] = 0.f;
     }
 
-    const int kv_end = causal ? min(m, q0 + kTile) : m;
+    const int mk = keys_valid(key_len, int(bh), H, m);     // keys past mk: padding
+    const int kv_end = causal ? min(mk, q0 + kTile) : mk;
     for (int k0 = 0; k0 < kv_end; k0 += kTile) {
         __syncthreads();
         for (int idx = threadIdx.x; idx < kTile * d; idx += kThreads) {
@@ -101,8 +104,8 @@ fwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict
                 s1 = fmaf(q, Ks[(lane + 32) * pk + c], s1);
             }
             const int j0 = k0 + lane, j1 = k0 + lane + 32;
-            s0 = (j0 < m && !(causal && j0 > i)) ? s0 * scale : -INFINITY;
-            s1 = (j1 < m && !(causal && j1 > i)) ? s1 * scale : -INFINITY;
+            s0 = (j0 < mk && !(causal && j0 > i)) ? s0 * scale : -INFINITY;
+            s1 = (j1 < mk && !(causal && j1 > i)) ? s1 * scale : -INFINITY;
             const float mnew = fmaxf(mrow[rr], warp_max(fmaxf(s0, s1)));
             if (mnew == -INFINITY) continue;  // whole row masked so far
             const float alpha = expf(mrow[rr] - mnew);
@@ -156,7 +159,7 @@ bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict
            const T* __restrict__ dO, const float* __restrict__ LSE,
            const float* __restrict__ Dd, int d_pitch, float* __restrict__ dQacc,
            T* __restrict__ dK, T* __restrict__ dV, int n, int m, int d, int dv, int causal,
-           float scale) {
+           float scale, const int* __restrict__ key_len, int H) {
     extern __shared__ float sm[];
     const int pq = odd_pitch(d), po = odd_pitch(dv);
     float* Ks = sm;                          // [64][d]
@@ -190,6 +193,7 @@ bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict
 #pragma unroll
         for (int k = 0; k < kCols; ++k) accK[rr][k] = accV[rr][k] = 0.f;
 
+    const int mk = keys_valid(key_len, int(bh), H, m);     // keys past mk: padding
     const int q_begin = causal ? k0 : 0;  // queries before the block see none of its keys
     for (int q0 = q_begin; q0 < n; q0 += kTile) {
         __syncthreads();
@@ -226,8 +230,8 @@ bwd_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __restrict
                 t1 = fmaf(vc, dOs[(lane + 32) * po + c], t1);
             }
             const int i0 = q0 + lane, i1 = q0 + lane + 32;
-            const bool ok0 = j < m && i0 < n && !(causal && j > i0);
-            const bool ok1 = j < m && i1 < n && !(causal && j > i1);
+            const bool ok0 = j < mk && i0 < n && !(causal && j > i0);
+            const bool ok1 = j < mk && i1 < n && !(causal && j > i1);
             const float p0 = ok0 ? expf(s0 * scale - lse_s[lane]) : 0.f;
             const float p1 = ok1 ? expf(s1 * scale - lse_s[lane + 32]) : 0.f;
             const float ds0 = p0 * (t0 - D_s[lane]);

@@ -10,6 +10,10 @@ workload's seed draws Q, K, V and dO, in that order, as fp32 standard normals
 scaled by each tensor's standard deviation. For a bf16 workload every tensor
 is then rounded to bf16, and both the GPU path and the float64 oracle see
 exactly those rounded values, so input quantisation is never counted as error.
+
+Padded workloads also carry the number of valid keys of each batch element
+(the key padding mask): either listed, or drawn uniformly from
+[pad_min, m] by a generator seeded with seed + 7919.
 """
 from __future__ import annotations
 
@@ -36,6 +40,32 @@ class Workload:
     std_qk: float = 1.0
     std_vo: float = 1.0
     doc: str = ""
+    pad_min: int = 0                 # > 0: key lengths drawn from [pad_min, m]
+    lengths: tuple | None = None     # explicit key lengths, one per batch element
+
+    def key_len(self):
+        """Valid keys per batch element (list of B ints), or None unpadded."""
+        if self.lengths is not None:
+            return [int(x) for x in self.lengths]
+        if self.pad_min <= 0:
+            return None
+        g = torch.Generator().manual_seed(self.seed + 7919)
+        return [int(x) for x in torch.randint(self.pad_min, self.m + 1, (self.B,), generator=g)]
+
+    def _pairs(self) -> float:
+        """Unmasked (query, key) pairs summed over the batch, per head. The
+        unpadded count keeps the n*m/2 convention for causal workloads."""
+        kl = self.key_len()
+        if kl is None:
+            p = self.B * self.n * self.m
+            return p / 2.0 if self.causal else float(p)
+        total = 0
+        for L in kl:
+            if self.causal:
+                total += sum(min(i + 1, L) for i in range(self.n))
+            else:
+                total += self.n * L
+        return float(total)
 
     @property
     def scale(self) -> float:
@@ -43,13 +73,21 @@ class Workload:
         return 1.0 / math.sqrt(self.d)
 
     def bwd_flops(self) -> float:
-        """Counted backward FLOPs: 2.5x the forward's two matmuls, halved when causal."""
-        f = 2.5 * 4.0 * self.B * self.H * self.n * self.m * self.d
-        return f / 2.0 if self.causal else f
+        """Counted backward FLOPs: 2.5x the forward's two matmuls, halved when
+        causal; with a padding mask, over the unmasked pairs only."""
+        return 2.5 * 4.0 * self.H * self.d * self._pairs()
 
     def fwd_flops(self) -> float:
-        f = 4.0 * self.B * self.H * self.n * self.m * self.d
-        return f / 2.0 if self.causal else f
+        return 4.0 * self.H * self.d * self._pairs()
+
+    def head_bwd_flops(self, b: int) -> float:
+        """Counted backward FLOPs of one (batch element b, head) problem."""
+        kl = self.key_len()
+        if kl is None:
+            return self.bwd_flops() / (self.B * self.H)
+        L = kl[b]
+        pairs = sum(min(i + 1, L) for i in range(self.n)) if self.causal else self.n * L
+        return 2.5 * 4.0 * self.d * pairs
 
 
 WORKLOADS = {
@@ -69,6 +107,10 @@ WORKLOADS = {
     "causal_b4h16_n1024_d64_f32": Workload(
         "causal_b4h16_n1024_d64_f32", 4, 16, 1024, 1024, 64, 64, "f32", True, 6,
         doc="B=4 H=16 N=1024 d=64 fp32 causal (the fp32 tensor-core path)"),
+    "padded_b8h16_n1024_d64": Workload(
+        "padded_b8h16_n1024_d64", 8, 16, 1024, 1024, 64, 64, "bf16", False, 7, pad_min=128,
+        doc="B=8 H=16 N=1024 d=64 bf16 with a key padding mask: valid keys per batch "
+            "element uniform in [128, 1024]"),
     "causal_b1h32_n16384_d128": Workload(
         "causal_b1h32_n16384_d128", 1, 32, 16384, 16384, 128, 128, "bf16", True, 5,
         doc="long context B=1 H=32 N=16384 d=128 bf16 causal"),
@@ -98,7 +140,10 @@ def make_inputs(w: Workload, seed: int | None = None):
 
 
 def make_small(B, H, n, m, d, dv, dtype="bf16", causal=False, seed=0,
-               std_qk=1.0, std_vo=1.0) -> Workload:
-    """An ad-hoc workload for tests (ragged and edge shapes)."""
-    return Workload(f"adhoc_{B}x{H}x{n}x{m}x{d}x{dv}_{dtype}_{int(causal)}_{seed}",
-                    B, H, n, m, d, dv, dtype, causal, seed, std_qk, std_vo)
+               std_qk=1.0, std_vo=1.0, lengths=None) -> Workload:
+    """An ad-hoc workload for tests (ragged and edge shapes); ``lengths``:
+    optional key lengths, one per batch element."""
+    tag = "" if lengths is None else "_pad" + "-".join(str(int(x)) for x in lengths)
+    return Workload(f"adhoc_{B}x{H}x{n}x{m}x{d}x{dv}_{dtype}_{int(causal)}_{seed}{tag}",
+                    B, H, n, m, d, dv, dtype, causal, seed, std_qk, std_vo,
+                    lengths=None if lengths is None else tuple(int(x) for x in lengths))

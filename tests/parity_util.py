@@ -27,8 +27,11 @@ def gpu_run(w: synth.Workload, inputs=None):
     q, k, v, do = synth.make_inputs(w) if inputs is None else inputs
     dev = torch.device("cuda:0")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o, lse = lib.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale)
-    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, dod, lse, causal=w.causal, scale=w.scale)
+    kl = w.key_len()
+    kl_t = None if kl is None else torch.tensor(kl, dtype=torch.int32, device=dev)
+    o, lse = lib.attn_fwd(qd, kd, vd, causal=w.causal, scale=w.scale, key_len=kl_t)
+    dq, dk, dv = lib.attn_bwd(qd, kd, vd, o, dod, lse, causal=w.causal, scale=w.scale,
+                              key_len=kl_t)
     torch.cuda.synchronize()
     assert lib.attn_get_device_error() == 0
     return (q, k, v, do), (o, lse, dq, dk, dv)
@@ -38,8 +41,9 @@ def full_compare(w: synth.Workload):
     """Every element of O, LSE, dQ, dK, dV against the float64 oracle."""
     (q, k, v, do), outs = gpu_run(w)
     Q, K, V, dO = (t.to(torch.float64).numpy() for t in (q, k, v, do))
-    O, lse = ref.attention_forward(Q, K, V, w.causal, w.scale)
-    dQ, dK, dV = ref.attention_backward(Q, K, V, dO, w.causal, w.scale)
+    kl = w.key_len()
+    O, lse = ref.attention_forward(Q, K, V, w.causal, w.scale, key_len=kl)
+    dQ, dK, dV = ref.attention_backward(Q, K, V, dO, w.causal, w.scale, key_len=kl)
     errs = {}
     for name, g, r in zip(("O", "LSE", "dQ", "dK", "dV"), outs, (O, lse, dQ, dK, dV)):
         assert tuple(g.shape) == r.shape, name
@@ -55,8 +59,9 @@ def heads_compare(w: synth.Workload, heads):
     errs = {name: 0.0 for name in ("O", "LSE", "dQ", "dK", "dV")}
     for (b, h) in heads:
         Qh, Kh, Vh, dOh = (t[b, h].to(torch.float64).numpy() for t in (q, k, v, do))
-        O_r, lse_r = ref.head_forward(Qh, Kh, Vh, w.causal, w.scale)
-        dQ_r, dK_r, dV_r = ref.head_backward(Qh, Kh, Vh, dOh, w.causal, w.scale)
+        L = None if w.key_len() is None else w.key_len()[b]
+        O_r, lse_r = ref.head_forward(Qh, Kh, Vh, w.causal, w.scale, key_len=L)
+        dQ_r, dK_r, dV_r = ref.head_backward(Qh, Kh, Vh, dOh, w.causal, w.scale, key_len=L)
         got = {"O": o[b, h], "LSE": lse[b, h], "dQ": dq[b, h], "dK": dk[b, h], "dV": dv[b, h]}
         want = {"O": O_r, "LSE": lse_r, "dQ": dQ_r, "dK": dK_r, "dV": dV_r}
         for name in errs:

@@ -167,3 +167,19 @@ def test_argument_checks_output_projection(L):
     r = lambda x: -(-x // 256) * 256
     assert L.attn_outproj_bwd_workspace_size(2, 64, 64, 2, 64, 1) == 2 * r(2 * 64 * 2 * 64 * 2)
     assert L.attn_outproj_bwd_workspace_size(2, 64, 64, 2, 64, 0) == 0
+
+
+def test_argument_checks_masked(L):
+    """The padding-mask calls check like attn_fwd / attn_bwd, plus key_len's
+    4-byte alignment; a NULL key_len is the unmasked call."""
+    kl_mis = ctypes.c_void_p(0x10002)
+    assert L.lib.attn_fwd_masked(P, P, P, P, P, kl_mis, 1, 1, 64, 64, 64, 64, 1, 0, 0.125, NUL) == 5
+    assert L.lib.attn_fwd_masked(NUL, P, P, P, P, P, 1, 1, 64, 64, 64, 64, 1, 0, 0.125, NUL) == 1
+    assert L.lib.attn_fwd_masked(P, P, P, P, P, P, 1, 1, 64, 65, 64, 64, 1, 1, 0.125, NUL) == 2
+    need = L.attn_bwd_workspace_size(1, 1, 64, 64, 64, 64, 1)
+    assert L.lib.attn_bwd_masked(P, P, P, P, P, P, kl_mis, P, P, P, P, need, 1, 1, 64, 64, 64, 64,
+                                 1, 0, 0.125, NUL) == 5
+    assert L.lib.attn_bwd_masked(P, P, P, P, P, P, P, P, P, P, P, need - 1, 1, 1, 64, 64, 64, 64,
+                                 1, 0, 0.125, NUL) == 6
+    if not torch.cuda.is_available():
+        assert L.lib.attn_fwd_masked(P, P, P, P, P, NUL, 1, 1, 64, 64, 64, 64, 1, 0, 0.125, NUL) == 7
