@@ -292,13 +292,11 @@ def run_ours(args, w, rank, world, local):
     peaks, peaks_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_note = f"bf16_tflops ({peaks_src}, burst)"
-    if "bwd_f32x_kv" in by_kernel:
+    if "bwd_f32x" in by_kernel:
         # fp32 by bf16 pieces: six bf16 MMAs per fp32 product, so the peak is
-        # a sixth of the bf16 one. The dK/dV pass does four of the five
-        # contractions of the counted FLOPs (S^T, dP^T, dV, dK); the dQ pass
-        # does dQ and recomputes S and dP, which the count does not credit.
-        main = max(("bwd_f32x_kv", "bwd_f32x_dq"), key=lambda k2: statistics.mean(by_kernel[k2]))
-        share = 0.8 if main == "bwd_f32x_kv" else 0.2
+        # a sixth of the bf16 one. The one launch runs both passes (the dQ
+        # pass recomputes S and dP, which the count does not credit).
+        main, share = "bwd_f32x", 1.0
         peak, peak_note = peak / 6.0, f"bf16_tflops / 6 ({peaks_src}, burst)"
     else:
         main = "bwd_tensor" if "bwd_tensor" in by_kernel else "bwd_simt"

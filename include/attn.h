@@ -217,8 +217,7 @@ typedef enum {
     ATTN_KERNEL_PROJ_GATHER = 7,  /* per-head gradients / weights side by side */
     ATTN_KERNEL_GEMM = 8,         /* tcgen05 GEMM of the projection gradients  */
     ATTN_KERNEL_FWD_F32X = 9,     /* tcgen05 forward, fp32 by bf16 pieces      */
-    ATTN_KERNEL_BWD_F32X_KV = 10, /* ... backward pass for dK, dV              */
-    ATTN_KERNEL_BWD_F32X_DQ = 11  /* ... backward pass for dQ                  */
+    ATTN_KERNEL_BWD_F32X = 10     /* ... backward: dK/dV and dQ passes, one launch */
 } attn_kernel_id_t;
 
 typedef struct {

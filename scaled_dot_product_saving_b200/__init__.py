@@ -36,7 +36,7 @@ ATTN_ERR_DEVICE_TIMEOUT = 8
 
 KERNEL_NAMES = {1: "fwd_tensor", 2: "fwd_simt", 3: "preprocess", 4: "bwd_tensor",
                 5: "bwd_simt", 6: "finalize", 7: "proj_gather", 8: "gemm",
-                9: "fwd_f32x", 10: "bwd_f32x_kv", 11: "bwd_f32x_dq"}
+                9: "fwd_f32x", 10: "bwd_f32x"}
 
 
 class _KernelTime(ctypes.Structure):

@@ -389,26 +389,18 @@ attn_status_t bwd_f32x(const void* Q, const void* K, const void* V, const void* 
     attn_status_t s = f32x_grid(m, BH, &grid_kv);
     if (s == ATTN_OK) s = f32x_grid(n, BH, &grid_dq);
     if (s != ATTN_OK) return s;
-    if (cudaFuncSetAttribute(fx::bwd_kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fx::kKvSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(fx::bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fx::kDqSmemBytes) != cudaSuccess)
+    if (static_cast<unsigned long long>(grid_kv) + grid_dq > 0x7fffffffull) return ATTN_ERR_SHAPE;
+    if (cudaFuncSetAttribute(fx::bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fx::kBwdSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
-    const float* q = static_cast<const float*>(Q);
-    const float* k = static_cast<const float*>(K);
-    const float* v = static_cast<const float*>(V);
-    const float* g = static_cast<const float*>(dO);
-    s = traced(ATTN_KERNEL_BWD_F32X_KV, st, [&] {
-        fx::bwd_kv_kernel<<<grid_kv, fx::kBwdThreads, fx::kKvSmemBytes, st>>>(
-            q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dK), static_cast<float*>(dV), n, m,
-            d, dv, BH, causal, scale, scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
-        return launched();
-    });
-    if (s != ATTN_OK) return s;
-    return traced(ATTN_KERNEL_BWD_F32X_DQ, st, [&] {
-        fx::bwd_dq_kernel<<<grid_dq, fx::kBwdThreads, fx::kDqSmemBytes, st>>>(
-            q, k, v, g, lse2, Dd, n_pad, static_cast<float*>(dQ), n, m, d, dv, BH, causal, scale,
-            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
+    // One launch: the dK/dV pass's CTAs first, then the dQ pass's.
+    return traced(ATTN_KERNEL_BWD_F32X, st, [&] {
+        fx::bwd_kernel<<<grid_kv + grid_dq, fx::kBwdThreads, fx::kBwdSmemBytes, st>>>(
+            static_cast<const float*>(Q), static_cast<const float*>(K),
+            static_cast<const float*>(V), static_cast<const float*>(dO), lse2, Dd, n_pad,
+            static_cast<float*>(dQ), static_cast<float*>(dK), static_cast<float*>(dV), n, m, d, dv,
+            BH, causal, scale, scale * kLog2e, mask.key_len, mask.H, static_cast<int>(grid_kv),
+            kWaitBudgetNs);
         return launched();
     });
 }
@@ -584,7 +576,7 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const
                                     causal, scale, mask, st);
         if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, scale, st);
     }
-    if (s == ATTN_OK) g_last_launches = 3;
+    if (s == ATTN_OK) g_last_launches = (path == Path::kTensorF32x) ? 2 : 3;
     return s;
 }
 

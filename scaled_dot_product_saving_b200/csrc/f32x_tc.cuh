@@ -25,14 +25,15 @@
 // rows. Pieces of a tile are stored one after another, each in the 128-byte
 // swizzled layout the MMA descriptors read (rows of 64 bf16).
 //
-// Kernels (128 threads, one elected thread issues the MMAs, all threads load,
-// split and run the elementwise steps):
+// Kernels (one elected thread issues the MMAs, all threads load, split and
+// run the elementwise steps):
 //   fwd_kernel     a 128-query tile, 64-key tiles: S (SS), online softmax in
 //                  registers, P split into TMEM, P V (TS) added into O in
 //                  registers with the running rescale.
-//   bwd_kv_kernel  a 128-key tile, 64-query tiles: S^T, dP^T (SS), P^T and
+//   bwd_kernel     two passes in one launch (256 threads):
+//     kv_pass      a 128-key tile, 64-query tiles: S^T, dP^T (SS), P^T and
 //                  dS^T split into TMEM, dV += P^T dO and dK += dS^T Q (TS).
-//   bwd_dq_kernel  a 128-query tile, 64-key tiles: S, dP (SS), dS split into
+//     dq_pass      a 128-query tile, 64-key tiles: S, dP (SS), dS split into
 //                  TMEM, dQ += dS K (TS). dQ is written once, no atomics.
 // The backward is two passes that each recompute S and dP, so that neither
 // needs a transposed copy of dS in shared memory (three pieces of a 128 x 128
@@ -494,22 +495,22 @@ constexpr int kKvOffStage = kKvOffRow + 4 * kSmall * 4; // Q, dO, LSE | D of til
 constexpr int kKvOffBar = kKvOffStage + 2 * kStageBytes + 2 * kSmall * 4;
 constexpr int kKvSmemBytes = kKvOffBar + 128;
 
-// Grid: one CTA per (128-key tile, head), heads fastest; causal grids start
-// with the first key tiles (the most query tiles).
-__global__ void __launch_bounds__(kBwdThreads, 1)
-bwd_kv_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
-              const float* __restrict__ dO, const float* __restrict__ lse2,
-              const float* __restrict__ Dd, int n_pad, float* __restrict__ dK,
-              float* __restrict__ dV, int n, int m, int d, int dv, int BH, int causal, float scale,
-              float scale_log2, const int* __restrict__ key_len, int H,
-              unsigned long long budget_ns) {
+// CTA `cta` of the pass: one per (128-key tile, head), heads fastest; causal
+// passes start with the first key tiles (the most query tiles).
+__device__ __forceinline__ void
+kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+        const float* __restrict__ dO, const float* __restrict__ lse2,
+        const float* __restrict__ Dd, int n_pad, float* __restrict__ dK,
+        float* __restrict__ dV, int n, int m, int d, int dv, int BH, int causal, float scale,
+        float scale_log2, const int* __restrict__ key_len, int H,
+        unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kKvOffBar);
     float* sRow = reinterpret_cast<float*>(smem + kKvOffRow);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int lane128 = tid & 127, half = tid >> 7;
-    const int bh = int(blockIdx.x % unsigned(BH));
-    const int kt = int(blockIdx.x / unsigned(BH));
+    const int bh = cta % BH;
+    const int kt = cta / BH;
     const int k0 = kt * kBig, krow = k0 + lane128;
     const float* Qh = Q + size_t(bh) * n * d;
     const float* Kh = K + size_t(bh) * m * d;
@@ -668,20 +669,21 @@ constexpr int kDqOffStage = kDqOffV + 2 * kSmallTile;  // K, V of tile t + 2
 constexpr int kDqOffBar = kDqOffStage + 2 * kStageBytes;
 constexpr int kDqSmemBytes = kDqOffBar + 128;
 
-// Grid as the forward's.
-__global__ void __launch_bounds__(kBwdThreads, 1)
-bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
-              const float* __restrict__ dO, const float* __restrict__ lse2,
-              const float* __restrict__ Dd, int n_pad, float* __restrict__ dQ, int n, int m, int d,
-              int dv, int BH, int causal, float scale, float scale_log2,
-              const int* __restrict__ key_len, int H, unsigned long long budget_ns) {
+// CTA `cta` of the pass: one per (128-query tile, head), ordered as the
+// forward's CTAs.
+__device__ __forceinline__ void
+dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+        const float* __restrict__ dO, const float* __restrict__ lse2,
+        const float* __restrict__ Dd, int n_pad, float* __restrict__ dQ, int n, int m, int d,
+        int dv, int BH, int causal, float scale, float scale_log2,
+        const int* __restrict__ key_len, int H, unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kDqOffBar);
     const int tid = threadIdx.x, warp = tid >> 5;
     const int lane128 = tid & 127, half = tid >> 7;
     const int num_qt = (n + kBig - 1) / kBig;
-    const int bh = int(blockIdx.x % unsigned(BH));
-    const int rank = int(blockIdx.x / unsigned(BH));
+    const int bh = cta % BH;
+    const int rank = cta / BH;
     const int qt = causal ? num_qt - 1 - rank : rank;
     const int q0 = qt * kBig, row = q0 + lane128;
     const float* Qh = Q + size_t(bh) * n * d;
@@ -801,6 +803,28 @@ bwd_dq_kernel(const float* __restrict__ Q, const float* __restrict__ K, const fl
         record_device_error(kErrTimeout);
     }
     teardown(bars, tmem, kDqTmemCols, budget_ns);
+}
+
+// ------------------------------------------------------- one launch
+// Both passes in one grid: CTAs [0, kv_ctas) run the dK/dV pass and the rest
+// the dQ pass. The passes share no data, and one launch lets each pass's
+// last, partial wave of CTAs be filled by the other's.
+constexpr int kBwdSmemBytes = kKvSmemBytes > kDqSmemBytes ? kKvSmemBytes : kDqSmemBytes;
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+bwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
+           const float* __restrict__ dO, const float* __restrict__ lse2,
+           const float* __restrict__ Dd, int n_pad, float* __restrict__ dQ,
+           float* __restrict__ dK, float* __restrict__ dV, int n, int m, int d, int dv, int BH,
+           int causal, float scale, float scale_log2, const int* __restrict__ key_len, int H,
+           int kv_ctas, unsigned long long budget_ns) {
+    const int b = int(blockIdx.x);
+    if (b < kv_ctas)
+        kv_pass(b, Q, K, V, dO, lse2, Dd, n_pad, dK, dV, n, m, d, dv, BH, causal, scale,
+                scale_log2, key_len, H, budget_ns);
+    else
+        dq_pass(b - kv_ctas, Q, K, V, dO, lse2, Dd, n_pad, dQ, n, m, d, dv, BH, causal, scale,
+                scale_log2, key_len, H, budget_ns);
 }
 
 }  // namespace f32x
