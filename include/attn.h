@@ -65,8 +65,10 @@ typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype_t;
 
 /* Which kernels a call may use. ATTN_PATH_AUTO picks the tensor-core path
  * where it applies (bf16 with d == dv in {64, 128}; f32 with d, dv <= 64 and
- * multiples of 4) and the CUDA-core path otherwise. ATTN_PATH_SIMT forces the CUDA-core path. ATTN_PATH_TENSOR
- * requires the tensor-core path and makes other shapes ATTN_ERR_UNSUPPORTED.
+ * multiples of 4) and the CUDA-core path otherwise. ATTN_PATH_SIMT forces
+ * the CUDA-core path. ATTN_PATH_TENSOR requires the tensor-core path and
+ * makes other shapes ATTN_ERR_UNSUPPORTED. The CUDA-core path takes at most
+ * 65535 (batch, head) problems per call (ATTN_ERR_UNSUPPORTED beyond).
  * The setting is process-wide and applies to calls made after it. */
 typedef enum { ATTN_PATH_AUTO = 0, ATTN_PATH_SIMT = 1, ATTN_PATH_TENSOR = 2 } attn_path_t;
 

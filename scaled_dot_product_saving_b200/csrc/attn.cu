@@ -27,6 +27,7 @@ namespace {
 constexpr unsigned long long kWaitBudgetNs = 2000000000ull;   // 2 s per bounded wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTile = 128;
+constexpr int kSimtMaxHeads = 65535;   // the CUDA-core kernels put B*H in gridDim.y
 
 std::atomic<int> g_path{ATTN_PATH_AUTO};
 thread_local int g_last_launches = 0;
@@ -254,6 +255,7 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
     const int num_qt = (n + attn::fwdtc::kBM - 1) / attn::fwdtc::kBM;
     const int num_pairs = (num_qt + 1) / 2;
     const long long grid = static_cast<long long>(num_pairs) * BH;
+    if (grid > 0x7fffffffll) return ATTN_ERR_SHAPE;
     const int head_group = std::max(1, std::min(BH, 256 / num_pairs));
     return traced(ATTN_KERNEL_FWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::fwdtc::kThreads, C::kSmemBytes, st>>>(
@@ -343,6 +345,7 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     // per scheduling group: about 256 items a group.
     const int num_kt = (m + kTile - 1) / kTile;
     const long long items = static_cast<long long>(num_kt) * BH;
+    if (items > 0x7fffffffll) return ATTN_ERR_SHAPE;          // the kernel counts items in int
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     const int head_group = std::max(1, std::min(BH, 256 / num_kt));
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
@@ -496,6 +499,7 @@ attn_status_t attn_fwd_masked(const void* Q, const void* K, const void* V, void*
     Path path = Path::kSimt;
     if ((s = choose_path(dtype, d, dv, &path)) != ATTN_OK) return s;
     const int BH = B * H;
+    if (path == Path::kSimt && BH > kSimtMaxHeads) return ATTN_ERR_UNSUPPORTED;
     const Mask mask{key_len, H};
     cudaStream_t st = as_stream(stream);
     if (path == Path::kTensorF32x)
@@ -537,6 +541,7 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const
     Path path = Path::kSimt;
     if ((s = choose_path(dtype, d, dv, &path)) != ATTN_OK) return s;
     const bool tensor = path != Path::kSimt;
+    if (!tensor && static_cast<long long>(B) * H > kSimtMaxHeads) return ATTN_ERR_UNSUPPORTED;
 
     const int BH = B * H;
     const Mask mask{key_len, H};

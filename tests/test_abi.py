@@ -183,3 +183,15 @@ def test_argument_checks_masked(L):
                                  1, 0, 0.125, NUL) == 6
     if not torch.cuda.is_available():
         assert L.lib.attn_fwd_masked(P, P, P, P, P, NUL, 1, 1, 64, 64, 64, 64, 1, 0, 0.125, NUL) == 7
+
+
+def test_cuda_core_path_head_limit(L):
+    """The CUDA-core kernels put B*H in gridDim.y: more than 65535 problems
+    on that path are refused before any launch; the tensor-core paths take
+    them."""
+    assert fwd(L, dt=0, d=128, dv=128, B=65536, H=1) == 4      # fp32, width > 64: CUDA-core
+    assert fwd(L, d=40, dv=40, B=256, H=256) == 4             # bf16 odd width: CUDA-core
+    need = L.attn_bwd_workspace_size(65536, 1, 64, 64, 128, 128, 0)
+    assert bwd(L, dt=0, d=128, dv=128, B=65536, H=1, wsb=need) == 4
+    if not torch.cuda.is_available():
+        assert fwd(L, B=65536, H=1) == 7                       # bf16 d = 64: tensor cores
