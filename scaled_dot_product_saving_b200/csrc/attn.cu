@@ -375,7 +375,7 @@ attn_status_t fwd_f32x(const void* Q, const void* K, const void* V, void* O, flo
                              fx::kFwdSmemBytes) != cudaSuccess)
         return ATTN_ERR_CUDA;
     return traced(ATTN_KERNEL_FWD_F32X, st, [&] {
-        fx::fwd_kernel<<<grid, fx::kThreads, fx::kFwdSmemBytes, st>>>(
+        fx::fwd_kernel<<<grid, fx::kFwdThreads, fx::kFwdSmemBytes, st>>>(
             static_cast<const float*>(Q), static_cast<const float*>(K),
             static_cast<const float*>(V), static_cast<float*>(O), LSE, n, m, d, dv, BH, causal,
             scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);

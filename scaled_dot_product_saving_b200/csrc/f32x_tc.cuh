@@ -248,56 +248,48 @@ __device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem, uint32_t tme
     }
 }
 
-// Load 64 fp32 columns of this thread's TMEM lane at `taddr` (two 32-column
-// loads) into v.
-__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&v)[64]) {
-    uint32_t a[32], b[32];
-    tmem_ld32(taddr, a);
-    tmem_ld32(taddr + 32, b);
-    tmem_ld_wait(a);
-    tmem_ld_wait(b);
+// Columns [c0, c0 + 32) of a row, clipped to width (width, c0 multiples of 4).
+__device__ __forceinline__ void store_half(float* row, int c0, const float (&v)[32], int width) {
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-        v[c] = __uint_as_float(a[c]);
-        v[32 + c] = __uint_as_float(b[c]);
-    }
-}
-
-// Store columns [0, width) of a 64-wide fp32 row (width % 4 == 0).
-__device__ __forceinline__ void store_row(float* dst, const float (&v)[64], int width, float mul) {
-#pragma unroll
-    for (int c = 0; c < 64; c += 4)
-        if (c < width)
-            *reinterpret_cast<float4*>(dst + c) =
-                make_float4(v[c] * mul, v[c + 1] * mul, v[c + 2] * mul, v[c + 3] * mul);
+    for (int c = 0; c < 32; c += 4)
+        if (c0 + c < width)
+            *reinterpret_cast<float4*>(row + c0 + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
 }
 
 // ================================================================ forward
 // TMEM columns: S (64), P V of the current key tile (64), P pieces (96).
+// Two warpgroups: thread t owns row t % 128 and the key (and value) column
+// half t / 128 of it. The halves trade their row maxima through shared memory
+// once per key tile, so both apply the same running maximum and rescale, and
+// add up their row sums at the end.
+constexpr int kFwdThreads = 256;
 constexpr uint32_t kFwdColS = 0, kFwdColPV = 64, kFwdColP = 128, kFwdTmemCols = 256;
 constexpr int kFwdOffQ = 0;
 constexpr int kFwdOffK = kFwdOffQ + kBigTile;          // two buffers
 constexpr int kFwdOffV = kFwdOffK + 2 * kSmallTile;    // two buffers
 constexpr int kStageBytes = kSmall * 8 * 32;           // one fp32 64 x 64 tile in flight
 constexpr int kFwdOffStage = kFwdOffV + 2 * kSmallTile; // K, V of tile t + 2
-constexpr int kFwdOffBar = kFwdOffStage + 2 * kStageBytes;
+constexpr int kFwdOffX = kFwdOffStage + 2 * kStageBytes; // [2 halves][128 rows] floats
+constexpr int kFwdOffBar = kFwdOffX + 2 * kBig * 4;
 constexpr int kFwdSmemBytes = kFwdOffBar + 128;
 
 // Grid: one CTA per (128-query tile, head), heads fastest; causal grids start
 // with the last query tiles (the most key tiles).
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
 fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float* __restrict__ V,
            float* __restrict__ O, float* __restrict__ LSE, int n, int m, int d, int dv, int BH,
            int causal, float scale_log2, const int* __restrict__ key_len, int H,
            unsigned long long budget_ns) {
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + kFwdOffBar);
+    float* xch = reinterpret_cast<float*>(smem + kFwdOffX);
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int lane128 = tid & 127, half = tid >> 7;
     const int num_qt = (n + kBig - 1) / kBig;
     const int bh = int(blockIdx.x % unsigned(BH));
     const int rank = int(blockIdx.x / unsigned(BH));
     const int qt = causal ? num_qt - 1 - rank : rank;
-    const int q0 = qt * kBig, row = q0 + tid;
+    const int q0 = qt * kBig, row = q0 + lane128;
     const float* Qh = Q + size_t(bh) * n * d;
     const float* Kh = K + size_t(bh) * m * d;
     const float* Vh = V + size_t(bh) * m * dv;
@@ -308,8 +300,8 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     uint8_t* stK = smem + kFwdOffStage;
     uint8_t* stV = stK + kStageBytes;
     auto fetch_kv = [&](int t) {
-        fetch<kSmall, kThreads>(Kh, t * kSmall, m, d, stK, tid);
-        fetch<kSmall, kThreads>(Vh, t * kSmall, m, dv, stV, tid);
+        fetch<kSmall, kFwdThreads>(Kh, t * kSmall, m, d, stK, tid);
+        fetch<kSmall, kFwdThreads>(Vh, t * kSmall, m, dv, stV, tid);
         cp_async_commit();
     };
 
@@ -318,12 +310,12 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     if (aligned) {
         // Key tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
         if (T > 2) fetch_kv(2);
-        load_split<kBig, kThreads>(Qh, q0, n, d, smem + kFwdOffQ, tid);
-        load_split<kSmall, kThreads>(Kh, 0, m, d, smem + kFwdOffK, tid);
-        load_split<kSmall, kThreads>(Vh, 0, m, dv, smem + kFwdOffV, tid);
+        load_split<kBig, kFwdThreads>(Qh, q0, n, d, smem + kFwdOffQ, tid);
+        load_split<kSmall, kFwdThreads>(Kh, 0, m, d, smem + kFwdOffK, tid);
+        load_split<kSmall, kFwdThreads>(Vh, 0, m, dv, smem + kFwdOffV, tid);
         if (T > 1) {
-            load_split<kSmall, kThreads>(Kh, kSmall, m, d, smem + kFwdOffK + kSmallTile, tid);
-            load_split<kSmall, kThreads>(Vh, kSmall, m, dv, smem + kFwdOffV + kSmallTile, tid);
+            load_split<kSmall, kFwdThreads>(Kh, kSmall, m, d, smem + kFwdOffK + kSmallTile, tid);
+            load_split<kSmall, kFwdThreads>(Vh, kSmall, m, dv, smem + kFwdOffV + kSmallTile, tid);
         }
     }
     fence_proxy_async_smem();
@@ -331,7 +323,8 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t tl = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t tq = tmem + (uint32_t((warp & 3) * 32) << 16);   // this warp's lanes
+    const uint32_t tl = tq + 32 * half;                             // ... and column half
     const uint32_t sQ = smem_addr(smem + kFwdOffQ);
     const uint32_t sK = smem_addr(smem + kFwdOffK), sV = smem_addr(smem + kFwdOffV);
     const int never = 0;
@@ -342,54 +335,53 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
         mma6_ss(tmem + kFwdColS, sQ, kBigPiece, sK, kSmallPiece, kIdSS);
         mma_commit(&bars->bar_a);
     }
-    float o[64];
+    float o[32];
 #pragma unroll
-    for (int c = 0; c < 64; ++c) o[c] = 0.f;
-    float mrow = -INFINITY, lrow = 0.f;
+    for (int c = 0; c < 32; ++c) o[c] = 0.f;
+    float mrow = -INFINITY, lrow = 0.f;                  // lrow: this half's share of the sum
 
     for (int j = 0; ok && j < T; ++j) {
         const int buf = j & 1;
-        float alpha = 1.f;
+        const int kb = j * kSmall + 32 * half;            // first key of this half
+        float s[32];
+        float mx = -INFINITY;
         const bool got = mbar_wait_warp(&bars->bar_a, j & 1, &never, budget_ns);
         if (got) {
             tc_fence_after();
-            float s[64];
-            tmem_row64(tl + kFwdColS, s);
-            const int kb = j * kSmall;
-            float mx = -INFINITY;
+            uint32_t sr[32];
+            tmem_ld32(tl + kFwdColS, sr);
+            tmem_ld_wait(sr);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
+            for (int c = 0; c < 32; ++c) {
                 const int key = kb + c;
-                float x = s[c] * scale_log2;
+                float x = __uint_as_float(sr[c]) * scale_log2;
                 if (key >= mk || (causal && key > row)) x = -INFINITY;
                 s[c] = x;
                 mx = fmaxf(mx, x);
             }
-            const float mnew = fmaxf(mrow, mx);
-            const float base = (mnew == -INFINITY) ? 0.f : mnew;
-            alpha = (mrow == -INFINITY) ? 0.f : ex2(mrow - base);
-            float lsum = 0.f;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                s[c] = ex2(s[c] - base);
-                lsum += s[c];
-            }
-            lrow = lrow * alpha + lsum;
-            mrow = mnew;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                float v[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) v[c] = s[32 * h + c];
-                split_to_tmem(v, tl + kFwdColP + 16 * h);
-            }
-            tmem_st_wait();
         }
-        tc_fence_before();
+        xch[half * kBig + lane128] = mx;
         if (__syncthreads_or(!got)) {
             ok = false;
             break;
         }
+        // Both halves see the same two maxima, so mrow, base and alpha agree.
+        const float mnew = fmaxf(mrow, fmaxf(mx, xch[(half ^ 1) * kBig + lane128]));
+        const float base = (mnew == -INFINITY) ? 0.f : mnew;
+        const float alpha = (mrow == -INFINITY) ? 0.f : ex2(mrow - base);
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            s[c] = ex2(s[c] - base);
+            lsum += s[c];
+        }
+        lrow = lrow * alpha + lsum;
+        mrow = mnew;
+        // this half's 32 keys are K elements 32 half .. +31: columns 16 half ..
+        split_to_tmem(s, tq + kFwdColP + 16 * half);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncthreads();
         if (tid == 0) {
             tc_fence_after();
             mma6_ts(tmem + kFwdColPV, tmem + kFwdColP, sV + buf * kSmallTile, kIdTS, false);
@@ -403,16 +395,17 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
         const bool got2 = mbar_wait_warp(&bars->bar_b, j & 1, &never, budget_ns);
         if (got2) {
             tc_fence_after();
-            float pv[64];
-            tmem_row64(tl + kFwdColPV, pv);
+            uint32_t pv[32];
+            tmem_ld32(tl + kFwdColPV, pv);
+            tmem_ld_wait(pv);
 #pragma unroll
-            for (int c = 0; c < 64; ++c) o[c] = fmaf(o[c], alpha, pv[c]);
+            for (int c = 0; c < 32; ++c) o[c] = fmaf(o[c], alpha, __uint_as_float(pv[c]));
             // K_j (read by S_j) and V_j (read by P_j V_j) are free: split
             // tile j + 2 from the staging buffer into them, then start
             // fetching tile j + 3.
             if (j + 2 < T) {
-                split_staged<kSmall, kThreads>(stK, smem + kFwdOffK + buf * kSmallTile, tid);
-                split_staged<kSmall, kThreads>(stV, smem + kFwdOffV + buf * kSmallTile, tid);
+                split_staged<kSmall, kFwdThreads>(stK, smem + kFwdOffK + buf * kSmallTile, tid);
+                split_staged<kSmall, kFwdThreads>(stV, smem + kFwdOffV + buf * kSmallTile, tid);
                 fence_proxy_async_smem();
                 if (j + 3 < T) fetch_kv(j + 3);
             }
@@ -425,9 +418,17 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
     }
 
     if (ok) {
+        // The row sum is the two halves' shares added (in the same order in
+        // both halves).
+        xch[half * kBig + lane128] = lrow;
+        __syncthreads();
+        const float l = xch[lane128] + xch[kBig + lane128];
         if (row < n) {
-            store_row(O + (size_t(bh) * n + row) * dv, o, dv, 1.0f / lrow);
-            LSE[size_t(bh) * n + row] = (mrow + log2f(lrow)) * kLn2;
+            const float inv = 1.0f / l;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] *= inv;
+            store_half(O + (size_t(bh) * n + row) * dv, 32 * half, o, dv);
+            if (half == 0) LSE[size_t(bh) * n + row] = (mrow + log2f(l)) * kLn2;
         }
     } else if (tid == 0) {
         record_device_error(kErrTimeout);
@@ -473,13 +474,6 @@ __device__ __forceinline__ void add_tmem32(uint32_t taddr, float (&acc)[32]) {
     for (int c = 0; c < 32; ++c) acc[c] += __uint_as_float(r[c]);
 }
 
-// Columns [c0, c0 + 32) of a row, clipped to width (width, c0 multiples of 4).
-__device__ __forceinline__ void store_half(float* row, int c0, const float (&v)[32], int width) {
-#pragma unroll
-    for (int c = 0; c < 32; c += 4)
-        if (c0 + c < width)
-            *reinterpret_cast<float4*>(row + c0 + c) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
-}
 
 // ---------------------------------------------------- dK and dV pass
 // TMEM columns: S^T (64), dP^T (64), this tile's dV (64) and dK (64), P^T
