@@ -21,16 +21,18 @@
 //
 // Shapes. Operands are zero-padded to 64 columns, so d, dv <= 64 (multiples
 // of 4 for 16-byte loads). Every MMA is M = 128, N = 64, K = 16: the 128 rows
-// a CTA owns sit one per thread and TMEM lane, the streamed tiles have 64
-// rows. Pieces of a tile are stored one after another, each in the 128-byte
-// swizzled layout the MMA descriptors read (rows of 64 bf16).
+// a CTA owns sit one per TMEM lane, the streamed tiles have 64 rows. Pieces
+// of a tile are stored one after another, each in the 128-byte swizzled
+// layout the MMA descriptors read (rows of 64 bf16).
 //
-// Kernels (one elected thread issues the MMAs, all threads load, split and
-// run the elementwise steps):
+// Kernels (256 threads; thread t owns row t % 128 and the column half t / 128
+// of it; one elected thread issues the MMAs, all threads load, split and run
+// the elementwise steps):
 //   fwd_kernel     a 128-query tile, 64-key tiles: S (SS), online softmax in
-//                  registers, P split into TMEM, P V (TS) added into O in
+//                  registers (the halves trade row maxima through shared
+//                  memory), P split into TMEM, P V (TS) added into O in
 //                  registers with the running rescale.
-//   bwd_kernel     two passes in one launch (256 threads):
+//   bwd_kernel     two passes in one launch:
 //     kv_pass      a 128-key tile, 64-query tiles: S^T, dP^T (SS), P^T and
 //                  dS^T split into TMEM, dV += P^T dO and dK += dS^T Q (TS).
 //     dq_pass      a 128-query tile, 64-key tiles: S, dP (SS), dS split into
@@ -51,7 +53,6 @@
 namespace attn {
 namespace f32x {
 
-constexpr int kThreads = 128;
 constexpr int kBig = 128;                       // rows a CTA owns (= threads = TMEM lanes)
 constexpr int kSmall = 64;                      // rows of a streamed tile
 constexpr int kWidth = 64;                      // padded operand width
