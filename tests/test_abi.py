@@ -195,3 +195,13 @@ def test_cuda_core_path_head_limit(L):
     assert bwd(L, dt=0, d=128, dv=128, B=65536, H=1, wsb=need) == 4
     if not torch.cuda.is_available():
         assert fwd(L, B=65536, H=1) == 7                       # bf16 d = 64: tensor cores
+
+
+def test_kernel_names_match_the_header(L):
+    """Every kernel id attn.h declares has a name in the binding's table used
+    by the tracer, and no name is left over."""
+    text = open(HEADER).read()
+    body = text[text.index("typedef enum {", text.index("ATTN_KERNEL_FWD_TENSOR") - 200):]
+    body = body[:body.index("attn_kernel_id_t")]
+    ids = {int(v) for v in re.findall(r"ATTN_KERNEL_[A-Z0-9_]+\s*=\s*(\d+)", body)}
+    assert ids == set(L.KERNEL_NAMES), (ids, sorted(L.KERNEL_NAMES))
