@@ -9,14 +9,21 @@ when causal) over the backward's device time, in TFLOP/s, summed over ranks.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
     python bench.py --impl reference ...     # the float64 CPU oracle, timed
 
-With N > 1 the script runs under torch.distributed.run, one rank per GPU; the
-(batch, head) problems are independent, so every rank runs the same workload
-on its own seeded data with no collective on the data path ("weak" scaling),
-and the timed region is bracketed by barriers and reduced as a max over ranks.
+With N > 1 the script runs under torch.distributed.run, one rank per GPU. The
+(batch, head) problems are independent, so there is no collective on the data
+path in either of the two ways of spreading work over ranks:
+  --split replicas (default)  every rank runs the whole workload on its own
+                              seeded data ("weak" scaling);
+  --split heads               the ranks share one workload: rank r takes a
+                              contiguous slice of its B*H problems, the same
+                              inputs the 1-GPU run sees ("strong" scaling).
+The timed region is bracketed by barriers and reduced as a max over ranks;
+`value` is all ranks' counted FLOPs over the slowest rank's time.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -57,6 +64,11 @@ def parse_args(argv=None):
                    help="kernel path the library may use (attn_set_path)")
     p.add_argument("--proj", action="store_true",
                    help="time attn_proj_bwd (projection and input gradients) instead")
+    p.add_argument("--dq-path", choices=["auto", "reduce", "separate"], default="auto",
+                   help="how the bf16 tensor-core backward computes dQ (attn_set_dq_path)")
+    p.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                   help="replicas: every rank runs the whole workload; heads: the ranks "
+                        "share the workload's (batch, head) problems")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -221,6 +233,63 @@ def aggregate(per_rank_flops, local_ms, world, device):
     return world * per_rank_flops / (slowest_ms * 1e-3) / 1e12, slowest_ms
 
 
+def sum_over_ranks(value, world, device):
+    if world == 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_slice(problems, rank, world):
+    """Rank `rank`'s contiguous share [lo, hi) of `problems` (batch, head)
+    problems numbered b*H + h; the shares of all ranks tile [0, problems)."""
+    return problems * rank // world, problems * (rank + 1) // world
+
+
+def slice_runs(B, H, lo, hi):
+    """Problems [lo, hi) as runs the library takes in one call each, as
+    (b0, nb, h0, nh): whole batch elements b0..b0+nb-1 (h0 = 0, nh = H), or
+    heads h0..h0+nh-1 of the single batch element b0 (nb = 1)."""
+    runs, p = [], lo
+    while p < hi:
+        b, h = divmod(p, H)
+        if h == 0 and hi - p >= H:
+            nb = (hi - p) // H
+            runs.append((b, nb, 0, H))
+            p += nb * H
+        else:
+            nh = min(H - h, hi - p)
+            runs.append((b, 1, h, nh))
+            p += nh
+    return runs
+
+
+def run_flops(w, run):
+    """Counted backward FLOPs of one run of problems."""
+    b0, nb, _, nh = run
+    return sum(nh * w.head_bwd_flops(b) for b in range(b0, b0 + nb))
+
+
+def make_parts(w, split, rank, world):
+    """The CPU inputs this rank works on, as a list of parts: (sub-workload,
+    (q, k, v, do), key lengths or None, counted backward FLOPs). A part is one
+    attn_fwd + attn_bwd call."""
+    if split == "replicas":
+        return [(w, synth.make_inputs(w, seed=w.seed + 1000 * rank), w.key_len(), w.bwd_flops())]
+    q, k, v, do = synth.make_inputs(w)               # the 1-GPU run's inputs
+    kl = w.key_len()
+    parts = []
+    for run in slice_runs(w.B, w.H, *rank_slice(w.B * w.H, rank, world)):
+        b0, nb, h0, nh = run
+        sub = dataclasses.replace(w, name=f"{w.name}[b{b0}:{b0 + nb},h{h0}:{h0 + nh}]", B=nb, H=nh,
+                                  lengths=None if kl is None else tuple(kl[b0:b0 + nb]), pad_min=0)
+        ts = tuple(t[b0:b0 + nb, h0:h0 + nh].contiguous() for t in (q, k, v, do))
+        parts.append((sub, ts, None if kl is None else kl[b0:b0 + nb], run_flops(w, run)))
+    return parts
+
+
 # ---------------------------------------------------------------- our arm
 def run_ours(args, w, rank, world, local):
     import scaled_dot_product_saving_b200 as lib
@@ -229,15 +298,38 @@ def run_ours(args, w, rank, world, local):
     torch.cuda.set_device(dev)
     lib.attn_set_path({"auto": lib.ATTN_PATH_AUTO, "simt": lib.ATTN_PATH_SIMT,
                        "tensor": lib.ATTN_PATH_TENSOR}[args.path])
-    q, k, v, do = (t.to(dev) for t in synth.make_inputs(w, seed=w.seed + 1000 * rank))
-    kl_list = w.key_len()
-    kl = None if kl_list is None else torch.tensor(kl_list, dtype=torch.int32, device=dev)
-    o = torch.empty((w.B, w.H, w.n, w.dv), dtype=q.dtype, device=dev)
-    lse = torch.empty((w.B, w.H, w.n), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(lib.attn_bwd_workspace_size(w.B, w.H, w.n, w.m, w.d, w.dv, q.dtype),
-                     dtype=torch.uint8, device=dev)
-    working_set = sum(t.numel() * t.element_size() for t in (q, k, v, o, do, dq, dk, dv, ws))
+    lib.attn_set_dq_path({"auto": lib.ATTN_DQ_AUTO, "reduce": lib.ATTN_DQ_REDUCE,
+                          "separate": lib.ATTN_DQ_SEPARATE}[args.dq_path])
+
+    # Device buffers of every part (one attn_fwd + attn_bwd call each).
+    class Part:
+        def __init__(self, sub, cpu, kl_list, flops):
+            self.w, self.flops = sub, flops
+            self.q, self.k, self.v, self.do = (t.to(dev) for t in cpu)
+            self.kl = None if kl_list is None else torch.tensor(kl_list, dtype=torch.int32,
+                                                                device=dev)
+            self.o = torch.empty((sub.B, sub.H, sub.n, sub.dv), dtype=self.q.dtype, device=dev)
+            self.lse = torch.empty((sub.B, sub.H, sub.n), dtype=torch.float32, device=dev)
+            self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.q, self.k, self.v))
+            self.ws = torch.empty(lib.attn_bwd_workspace_size(sub.B, sub.H, sub.n, sub.m, sub.d,
+                                                              sub.dv, self.q.dtype),
+                                  dtype=torch.uint8, device=dev)
+
+        def tensors(self):
+            return (self.q, self.k, self.v, self.o, self.do, self.dq, self.dk, self.dv, self.ws)
+
+        def fwd(self, stream=None):
+            lib.attn_fwd(self.q, self.k, self.v, causal=self.w.causal, scale=self.w.scale,
+                         out=self.o, lse=self.lse, key_len=self.kl, stream=stream)
+
+        def bwd(self, stream=None):
+            lib.attn_bwd(self.q, self.k, self.v, self.o, self.do, self.lse, causal=self.w.causal,
+                         scale=self.w.scale, workspace=self.ws, dq=self.dq, dk=self.dk,
+                         dv=self.dv, key_len=self.kl, stream=stream)
+
+    parts = [Part(*p) for p in make_parts(w, args.split, rank, world)]
+    local_flops = sum(p.flops for p in parts)
+    working_set = sum(t.numel() * t.element_size() for p in parts for t in p.tensors())
     flush = None
     if working_set < 2 * L2_BYTES:
         flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
@@ -247,11 +339,12 @@ def run_ours(args, w, rank, world, local):
             flush.zero_()
         if evs:
             evs[0].record()
-        lib.attn_fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, key_len=kl)
+        for p in parts:
+            p.fwd()
         if evs:
             evs[1].record()
-        lib.attn_bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws,
-                     dq=dq, dk=dk, dv=dv, key_len=kl)
+        for p in parts:
+            p.bwd()
         if evs:
             evs[2].record()
 
@@ -267,7 +360,7 @@ def run_ours(args, w, rank, world, local):
     barrier(world, local)
     torch.cuda.synchronize()
     sampler.start()
-    lib.attn_trace_begin(min(65536, 8 * args.steps))
+    lib.attn_trace_begin(min(65536, 8 * len(parts) * args.steps))
     t_start.record()
     for s in range(args.steps):
         step(evs[s])
@@ -284,7 +377,9 @@ def run_ours(args, w, rank, world, local):
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
     bwd_sum, fwd_sum = sum(bwd_ms), sum(fwd_ms)
     slow_total, slow_bwd, slow_fwd = max_over_ranks([total_ms, bwd_sum, fwd_sum], world, dev)
-    value = world * args.steps * w.bwd_flops() / (slow_bwd * 1e-3) / 1e12
+    job_flops = sum_over_ranks(local_flops, world, dev)            # backward FLOPs of one step
+    job_fwd_flops = job_flops * w.fwd_flops() / w.bwd_flops()
+    value = args.steps * job_flops / (slow_bwd * 1e-3) / 1e12
 
     by_kernel = {}
     for name, ms in trace:
@@ -292,17 +387,28 @@ def run_ours(args, w, rank, world, local):
     peaks, peaks_src = measured_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_note = f"bf16_tflops ({peaks_src}, burst)"
+    # FLOPs each backward kernel performs, as a share of the counted backward
+    # FLOPs (five contractions): the fused kernel all five; the separate dK/dV
+    # pass four (S, dP, dV, dK) and the dQ pass three (S and dP again, dQ).
+    share = {"bwd_tensor": 1.0, "bwd_simt": 1.0, "bwd_f32x": 1.0, "bwd_kv": 0.8, "bwd_dq": 0.6}
     if "bwd_f32x" in by_kernel:
         # fp32 by bf16 pieces: six bf16 MMAs per fp32 product, so the peak is
         # a sixth of the bf16 one. The one launch runs both passes (the dQ
         # pass recomputes S and dP, which the count does not credit).
-        main, share = "bwd_f32x", 1.0
+        main = "bwd_f32x"
         peak, peak_note = peak / 6.0, f"bf16_tflops / 6 ({peaks_src}, burst)"
+    elif "bwd_kv" in by_kernel:
+        main = max(("bwd_kv", "bwd_dq"), key=lambda k2: sum(by_kernel[k2]))
     else:
         main = "bwd_tensor" if "bwd_tensor" in by_kernel else "bwd_simt"
-        share = 1.0
-    main_ms = statistics.mean(by_kernel[main])
-    achieved = share * w.bwd_flops() / (main_ms * 1e-3) / 1e12
+
+    def kernel_tflops(name):
+        # the kernel's own FLOPs per step over its device time per step
+        ms = statistics.mean(by_kernel[name]) * len(by_kernel[name]) / args.steps
+        return share[name] * local_flops / (ms * 1e-3) / 1e12
+    achieved = kernel_tflops(main)
+    per_kernel = {k2: {"tflops": round(kernel_tflops(k2), 3), "frac": round(kernel_tflops(k2) / peak, 4)}
+                  for k2 in by_kernel if k2 in share}
 
     # End to end through the public API with host buffers. Every step copies
     # its Q, K, V, dO in from pinned host memory, runs attn_fwd + attn_bwd and
@@ -311,20 +417,14 @@ def run_ours(args, w, rank, world, local):
     # step i's kernels, as a training loop feeding the library would.
     e2e = None
     if args.e2e_steps > 0:
-        ins = (q, k, v, do) if kl is None else (q, k, v, do, kl)
-        pin_in = [[t.to("cpu").pin_memory() for t in ins] for _ in range(2)]
-        pin_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (dq, dk, dv)]
-                   for _ in range(2)]
-        dev_sets = []
-        for b in range(2):
-            kl_b = kl if (kl is None or b == 0) else torch.empty_like(kl)
-            if b == 0:
-                dev_sets.append((q, k, v, do, o, lse, dq, dk, dv, ws, kl_b))
-            else:
-                dev_sets.append(tuple(torch.empty_like(t) for t in (q, k, v, do, o, lse, dq, dk, dv, ws))
-                                + (kl_b,))
-        h2d = sum(t.numel() * t.element_size() for t in pin_in[0])
-        d2h = sum(t.numel() * t.element_size() for t in pin_out[0])
+        sets = [parts, [Part(p.w, (p.q.cpu(), p.k.cpu(), p.v.cpu(), p.do.cpu()),
+                             None if p.kl is None else p.kl.tolist(), p.flops) for p in parts]]
+        pin_in = [[[t.to("cpu").pin_memory() for t in (p.q, p.k, p.v, p.do)
+                    + (() if p.kl is None else (p.kl,))] for p in parts] for _ in range(2)]
+        pin_out = [[[torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                     for t in (p.dq, p.dk, p.dv)] for p in parts] for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for pp in pin_in[0] for t in pp)
+        d2h = sum(t.numel() * t.element_size() for pp in pin_out[0] for t in pp)
         s_in, s_run, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
         ev_in = [torch.cuda.Event() for _ in range(2)]
         ev_run = [torch.cuda.Event() for _ in range(2)]
@@ -334,23 +434,24 @@ def run_ours(args, w, rank, world, local):
 
         def e2e_step(i):
             b = i % 2
-            qb, kb, vb, dob, ob, lseb, dqb, dkb, dvb, wsb, klb = dev_sets[b]
             s_in.wait_event(ev_free[b])
             with torch.cuda.stream(s_in):
-                dsts = (qb, kb, vb, dob) if klb is None else (qb, kb, vb, dob, klb)
-                for src, dst in zip(pin_in[b], dsts):
-                    dst.copy_(src, non_blocking=True)
+                for p, srcs in zip(sets[b], pin_in[b]):
+                    dsts = (p.q, p.k, p.v, p.do) + (() if p.kl is None else (p.kl,))
+                    for src, dst in zip(srcs, dsts):
+                        dst.copy_(src, non_blocking=True)
                 ev_in[b].record(s_in)
             s_run.wait_event(ev_in[b])
-            lib.attn_fwd(qb, kb, vb, causal=w.causal, scale=w.scale, out=ob, lse=lseb, stream=s_run,
-                         key_len=klb)
-            lib.attn_bwd(qb, kb, vb, ob, dob, lseb, causal=w.causal, scale=w.scale, workspace=wsb,
-                         dq=dqb, dk=dkb, dv=dvb, stream=s_run, key_len=klb)
+            for p in sets[b]:
+                p.fwd(stream=s_run)
+            for p in sets[b]:
+                p.bwd(stream=s_run)
             ev_run[b].record(s_run)
             s_out.wait_event(ev_run[b])
             with torch.cuda.stream(s_out):
-                for src, dst in zip((dqb, dkb, dvb), pin_out[b]):
-                    dst.copy_(src, non_blocking=True)
+                for p, dsts in zip(sets[b], pin_out[b]):
+                    for src, dst in zip((p.dq, p.dk, p.dv), dsts):
+                        dst.copy_(src, non_blocking=True)
                 ev_free[b].record(s_out)
 
         for i in range(2):                       # untimed: one round of both buffer sets
@@ -365,11 +466,18 @@ def run_ours(args, w, rank, world, local):
         if lib.attn_get_device_error() != 0:
             raise RuntimeError("device-side timeout in the end-to-end leg")
         (slow_e2e,) = max_over_ranks([ea.elapsed_time(eb)], world, dev)
-        e2e = {"value": round(world * args.e2e_steps * w.bwd_flops() / (slow_e2e * 1e-3) / 1e12, 3),
+        e2e = {"value": round(args.e2e_steps * job_flops / (slow_e2e * 1e-3) / 1e12, 3),
                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": round(slow_e2e / args.e2e_steps, 4),
                "pipelined": "2 buffer sets, upload/compute/download streams"}
 
+    kl_list = w.key_len()
+    if world == 1:
+        parallelism = "single GPU"
+    elif args.split == "heads":
+        parallelism = f"(batch, head) problems split over {world} ranks"
+    else:
+        parallelism = f"replicas: the whole workload on each of {world} ranks"
     result = {
         "metric": metric_for(w),
         "value": round(value, 3),
@@ -379,28 +487,30 @@ def run_ours(args, w, rank, world, local):
         "warmup": args.warmup,
         "ms_per_step": round(slow_total / args.steps, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.split == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": {
             "workload": w.name, "B": w.B, "H": w.H, "n": w.n, "m": w.m, "d": w.d, "dv": w.dv,
-            "causal": w.causal, "scale": w.scale, "path": args.path,
+            "causal": w.causal, "scale": w.scale, "path": args.path, "dq_path": args.dq_path,
             **({} if kl_list is None else {"key_len": kl_list}),
-            "parallelism": "replicas" if world == 1 else f"independent (batch, head) problems x{world}",
+            "parallelism": parallelism,
             "l2": ("flushed between steps (256 MiB write)" if flush is not None else
                    f"inputs larger than L2 ({working_set / 2**20:.0f} MiB per step)"),
         },
         "fwd_ms": round(slow_fwd / args.steps, 4),
         "bwd_ms": round(slow_bwd / args.steps, 4),
-        "fwd_tflops": round(world * args.steps * w.fwd_flops() / (slow_fwd * 1e-3) / 1e12, 3),
+        "fwd_tflops": round(args.steps * job_fwd_flops / (slow_fwd * 1e-3) / 1e12, 3),
         "frac_of_datasheet_bf16": round(value / world / DATASHEET_BF16_TFLOPS, 4),
         "kernel_ms": {k2: round(statistics.mean(v2), 4) for k2, v2 in by_kernel.items()},
         "roofline": {
             "bound": "tensor", "kernel": main, "achieved": round(achieved, 3),
             "peak": round(peak, 3), "peak_source": peak_note,
             "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "traffic": profiled_traffic(w.name),
+            "traffic": (profiled_traffic(w.name)
+                        if len(parts) == 1 and parts[0].w is w and main == "bwd_tensor" else None),
+            "kernels": per_kernel,
         },
         "e2e": e2e,
         "gpu_launches": len(trace),

@@ -69,8 +69,22 @@ typedef enum { ATTN_F32 = 0, ATTN_BF16 = 1 } attn_dtype_t;
  * the CUDA-core path. ATTN_PATH_TENSOR requires the tensor-core path and
  * makes other shapes ATTN_ERR_UNSUPPORTED. The CUDA-core path takes at most
  * 65535 (batch, head) problems per call (ATTN_ERR_UNSUPPORTED beyond).
- * The setting is process-wide and applies to calls made after it. */
+ * The setting belongs to the calling host thread (each thread starts with
+ * ATTN_PATH_AUTO) and applies to that thread's later calls, so threads that
+ * use different paths do not race on it. */
 typedef enum { ATTN_PATH_AUTO = 0, ATTN_PATH_SIMT = 1, ATTN_PATH_TENSOR = 2 } attn_path_t;
+
+/* How the bf16 tensor-core backward computes dQ ("Attention backward",
+ * Problem 5: dQ = scale * dS K, a sum over key tiles). ATTN_DQ_REDUCE: one
+ * key-tile-major kernel computes dK, dV and every partial dQ, and adds the
+ * partials into an fp32 accumulator in the workspace with TMA reduce-adds
+ * (converted to bf16 inside the same launch). ATTN_DQ_SEPARATE: a
+ * key-tile-major kernel computes dK and dV, then a query-tile-major kernel
+ * recomputes S and dP per query tile and sums dQ inside one CTA (seven
+ * contractions instead of five, no accumulator traffic). ATTN_DQ_AUTO picks
+ * the one measured faster. Results agree within rounding; the choice, like
+ * attn_path_t, belongs to the calling host thread. */
+typedef enum { ATTN_DQ_AUTO = 0, ATTN_DQ_REDUCE = 1, ATTN_DQ_SEPARATE = 2 } attn_dq_path_t;
 
 /*
  * attn_fwd -- O and LSE from Q, K, V.
@@ -88,9 +102,11 @@ attn_status_t attn_fwd(const void* Q, const void* K, const void* V,
 /*
  * attn_bwd_workspace_size -- bytes of device scratch that attn_bwd needs for
  * these sizes: D = rowsum(dO * O) and the LSE in base 2, both [B,H,n] fp32
- * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ
- * and 256 bytes for the work-item counter of the persistent tensor-core
- * backward (each region rounded up to 256 bytes).
+ * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ,
+ * then 256 bytes for two counters of the persistent tensor-core backward
+ * (its work items, and the dQ slabs its converter warps have claimed) and 4
+ * bytes per (batch, head) for the head's count of finished work items (each
+ * region rounded up to 256 bytes).
  * Returns 0 if the sizes are invalid.
  */
 size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv,
@@ -159,10 +175,15 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V,
  * exits. It allocates nothing and calls no allocating routine.
  *  - Sizes whose attn_bwd_workspace_size() exceeds the array are rejected
  *    with ATTN_ERR_WORKSPACE before anything is launched (the d = 64,
- *    B*H*n = 65536 problem fits; the long-context ones do not).
+ *    B*H*n = 65536 problem fits; the long-context ones do not). Argument
+ *    errors take precedence: the status is the one attn_bwd would give for
+ *    the same arguments without a workspace.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture on the device.
+ *    (cudaGetSymbolAddress, with that device current) and keeps it for as
+ *    long as that device's context lives; the first call after the context
+ *    has been replaced (cudaDeviceReset) looks it up again. Make those first
+ *    calls before any stream capture on the device. If the lookup fails the
+ *    call returns ATTN_ERR_CUDA, with the runtime's error state cleared.
  *  - Every call shares the one array, which keeps the last call's contents;
  *    the kernels rewrite what they read. Calls whose kernels overlap on the
  *    GPU (two streams, or two host threads) race on the array: serialise them.
@@ -215,11 +236,13 @@ typedef enum {
     ATTN_KERNEL_PREPROCESS = 3,   /* D = rowsum(dO*O), base-2 LSE, zero dQacc */
     ATTN_KERNEL_BWD_TENSOR = 4,   /* tcgen05 backward                         */
     ATTN_KERNEL_BWD_SIMT = 5,     /* CUDA-core backward                       */
-    ATTN_KERNEL_FINALIZE = 6,     /* dQ accumulator -> dQ                      */
+    ATTN_KERNEL_FINALIZE = 6,     /* dQ accumulator -> dQ (CUDA-core path)     */
     ATTN_KERNEL_PROJ_GATHER = 7,  /* per-head gradients / weights side by side */
     ATTN_KERNEL_GEMM = 8,         /* tcgen05 GEMM of the projection gradients  */
     ATTN_KERNEL_FWD_F32X = 9,     /* tcgen05 forward, fp32 by bf16 pieces      */
-    ATTN_KERNEL_BWD_F32X = 10     /* ... backward: dK/dV and dQ passes, one launch */
+    ATTN_KERNEL_BWD_F32X = 10,    /* ... backward: dK/dV and dQ passes, one launch */
+    ATTN_KERNEL_BWD_KV = 11,      /* tcgen05 dK/dV pass (ATTN_DQ_SEPARATE)      */
+    ATTN_KERNEL_BWD_DQ = 12       /* tcgen05 dQ pass (ATTN_DQ_SEPARATE)         */
 } attn_kernel_id_t;
 
 typedef struct {
@@ -281,11 +304,16 @@ attn_status_t attn_outproj_bwd(const void* O, const void* Wo, const void* G, voi
                                void* workspace, size_t workspace_bytes, int B, int n,
                                int d_model, int H, int dv, attn_dtype_t dtype, void* stream);
 
-/* Select the kernel path for later calls (see attn_path_t). */
+/* Select the kernel path for the calling thread's later calls (see
+ * attn_path_t). */
 attn_status_t attn_set_path(attn_path_t path);
 
-/* Number of kernels the last successful attn_fwd/attn_bwd/attn_proj_bwd/
- * attn_outproj_bwd call launched. */
+/* Select how the calling thread's later bf16 tensor-core backward calls
+ * compute dQ (see attn_dq_path_t). */
+attn_status_t attn_set_dq_path(attn_dq_path_t path);
+
+/* Number of kernels the calling thread's last successful attn_fwd/attn_bwd/
+ * attn_proj_bwd/attn_outproj_bwd call launched. */
 int attn_last_launch_count(void);
 
 /* A static, human-readable name for a status code. */

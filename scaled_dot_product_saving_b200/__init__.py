@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "AttnError", "LIB_PATH", "lib", "ATTN_F32", "ATTN_BF16",
     "ATTN_PATH_AUTO", "ATTN_PATH_SIMT", "ATTN_PATH_TENSOR",
+    "ATTN_DQ_AUTO", "ATTN_DQ_REDUCE", "ATTN_DQ_SEPARATE", "attn_set_dq_path",
     "attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_get_device_error",
     "attn_probe_timeout", "attn_set_path", "attn_last_launch_count", "attn_status_string",
     "dtype_code", "attn_trace_begin", "attn_trace_end", "KERNEL_NAMES",
@@ -31,12 +32,13 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 
 ATTN_F32, ATTN_BF16 = 0, 1
 ATTN_PATH_AUTO, ATTN_PATH_SIMT, ATTN_PATH_TENSOR = 0, 1, 2
+ATTN_DQ_AUTO, ATTN_DQ_REDUCE, ATTN_DQ_SEPARATE = 0, 1, 2
 ATTN_OK = 0
 ATTN_ERR_DEVICE_TIMEOUT = 8
 
 KERNEL_NAMES = {1: "fwd_tensor", 2: "fwd_simt", 3: "preprocess", 4: "bwd_tensor",
                 5: "bwd_simt", 6: "finalize", 7: "proj_gather", 8: "gemm",
-                9: "fwd_f32x", 10: "bwd_f32x"}
+                9: "fwd_f32x", 10: "bwd_f32x", 11: "bwd_kv", 12: "bwd_dq"}
 
 
 class _KernelTime(ctypes.Structure):
@@ -82,6 +84,8 @@ def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
     L.attn_probe_timeout.restype = i
     L.attn_set_path.argtypes = [i]
     L.attn_set_path.restype = i
+    L.attn_set_dq_path.argtypes = [i]
+    L.attn_set_dq_path.restype = i
     L.attn_last_launch_count.argtypes = []
     L.attn_last_launch_count.restype = i
     L.attn_status_string.argtypes = [i]
@@ -239,6 +243,10 @@ def attn_probe_timeout(timeout_us: int, stream=None) -> None:
 
 def attn_set_path(path: int) -> None:
     _check(lib.attn_set_path(int(path)), "attn_set_path")
+
+
+def attn_set_dq_path(path: int) -> None:
+    _check(lib.attn_set_dq_path(int(path)), "attn_set_dq_path")
 
 
 def attn_last_launch_count() -> int:

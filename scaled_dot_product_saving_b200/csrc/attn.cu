@@ -18,6 +18,8 @@
 #include "prep.cuh"
 #include "fwd_tc.cuh"
 #include "bwd_tc.cuh"
+#include "kv_tc.cuh"
+#include "dq_tc.cuh"
 #include "gemm_tc.cuh"
 #include "proj.cuh"
 #include "f32x_tc.cuh"
@@ -29,7 +31,11 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTile = 128;
 constexpr int kSimtMaxHeads = 65535;   // the CUDA-core kernels put B*H in gridDim.y
 
-std::atomic<int> g_path{ATTN_PATH_AUTO};
+// Per host thread: the kernel path a thread selected, and the launch count of
+// its last call (the trace state below is per thread too), so calls from
+// different threads never share mutable library state.
+thread_local int g_path = ATTN_PATH_AUTO;
+thread_local int g_dq_path = ATTN_DQ_AUTO;
 thread_local int g_last_launches = 0;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -62,7 +68,7 @@ bool f32x_path_fits(attn_dtype_t dtype, int d, int dv) {
 
 // Decide the path; ATTN_OK and *path set, or an error.
 attn_status_t choose_path(attn_dtype_t dtype, int d, int dv, Path* path) {
-    const int p = g_path.load();
+    const int p = g_path;
     const bool bf16 = tensor_path_fits(dtype, d, dv);
     const bool f32x = f32x_path_fits(dtype, d, dv);
     if (p == ATTN_PATH_TENSOR && !bf16 && !f32x) return ATTN_ERR_UNSUPPORTED;
@@ -79,10 +85,16 @@ struct Mask {
     int H;
 };
 
+// Backward workspace: base-2 LSE and D ([BH, n_pad] fp32 each), the fp32 dQ
+// accumulator [BH, n, d], then the tensor-core backwards' counters (int32):
+// work-item and converter-claim counters in the first 256 bytes, then one
+// count of landed work items per head. Every region starts on a 256-byte
+// boundary.
 struct Workspace {
-    size_t lse2_off, dd_off, dq_off, sched_off, total;
+    size_t lse2_off, dd_off, dq_off, cnt_off, n_counters, total;
     int n_pad;
 };
+
 
 Workspace carve(int B, int H, int n, int d) {
     Workspace w;
@@ -92,8 +104,9 @@ Workspace carve(int B, int H, int n, int d) {
     w.lse2_off = 0;
     w.dd_off = row_bytes;
     w.dq_off = 2 * row_bytes;
-    w.sched_off = w.dq_off + round_up(bh * static_cast<size_t>(n) * d * sizeof(float), 256);
-    w.total = w.sched_off + 256;   // the backward's work-item counter
+    w.cnt_off = w.dq_off + round_up(bh * static_cast<size_t>(n) * d * sizeof(float), 256);
+    w.n_counters = attn::bwdtc::kCntHeadBase + bh;
+    w.total = w.cnt_off + round_up(w.n_counters * sizeof(int), 256);
     return w;
 }
 
@@ -267,27 +280,28 @@ attn_status_t fwd_tensor(const void* Q, const void* K, const void* V, void* O, f
 
 template <typename T>
 attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float* lse2, float* Dd,
-                         float* dQacc, int* sched, int BH, int n, int n_pad, int d, int dv,
-                         float d_scale, bool zero_dq, cudaStream_t st) {
+                         float* dQacc, int* counters, size_t n_counters, int BH, int n, int n_pad,
+                         int d, int dv, float d_scale, bool zero_dq, cudaStream_t st) {
     const size_t rows = static_cast<size_t>(BH) * n_pad;
     const size_t dq_elems = zero_dq ? static_cast<size_t>(BH) * n * d : 0;
     const bool vec = sizeof(T) == 2 && dv % 8 == 0 && (dv / 8) <= 32 && 32 % (dv / 8) == 0 &&
                      dq_elems % 4 == 0;
     if (vec) {
-        const int rows_per_block = (attn::prep::kThreads / 32) * (32 / (dv / 8));
-        const int grid = grid_for(rows, rows_per_block, 148 * 16);
+        const int rows_per_block =
+            (attn::prep::kThreads / 32) * (32 / (dv / 8)) * attn::prep::kRowsInFlight;
+        const int grid = grid_for(rows, rows_per_block, sm_count() * 8);
         return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
             attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
-                lse2, Dd, dQacc, sched, dq_elems, BH, n, n_pad, dv, d_scale);
+                lse2, Dd, dQacc, counters, n_counters, dq_elems, BH, n, n_pad, dv, d_scale);
             return launched();
         });
     }
     const int grid = grid_for(rows, attn::prep::kThreads / 32, 148 * 16);
     return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
         attn::prep::preprocess_generic<T><<<grid, attn::prep::kThreads, 0, st>>>(
-            static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, sched,
-            dq_elems, BH, n, n_pad, dv, d_scale);
+            static_cast<const T*>(O), static_cast<const T*>(dO), LSE, lse2, Dd, dQacc, counters,
+            n_counters, dq_elems, BH, n, n_pad, dv, d_scale);
         return launched();
     });
 }
@@ -325,9 +339,9 @@ attn_status_t bwd_simt(const void* Q, const void* K, const void* V, const void* 
 
 template <int D>
 attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void* dO,
-                         const float* lse2, const float* Dd, int* sched, int n_pad, float* dQacc, void* dK,
-                         void* dV, int BH, int n, int m, int causal, float scale, Mask mask,
-                         cudaStream_t st) {
+                         const float* lse2, const float* Dd, int* counters, int n_pad, float* dQacc,
+                         void* dQ, void* dK, void* dV, int BH, int n, int m, int causal, float scale,
+                         Mask mask, cudaStream_t st) {
     using C = attn::bwdtc::Cfg<D>;
     CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
     if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) ||
@@ -350,10 +364,64 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     const int head_group = std::max(1, std::min(BH, 256 / num_kt));
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
         kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, sched, n_pad, n, m, BH, head_group, causal, scale,
+            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, counters, dQacc,
+            static_cast<__nv_bfloat16*>(dQ), n_pad, n, m, BH, head_group, causal, scale,
             scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
         return launched();
     });
+}
+
+// The bf16 backward as two passes (ATTN_DQ_SEPARATE): dK/dV key-tile major,
+// then dQ query-tile major, each persistent with one CTA per SM and its own
+// work counter.
+template <int D>
+attn_status_t bwd_separate(const void* Q, const void* K, const void* V, const void* dO,
+                           const float* lse2, const float* Dd, int* counters, int n_pad, void* dQ,
+                           void* dK, void* dV, int BH, int n, int m, int causal, float scale,
+                           Mask mask, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+    if (!make_map(&mq, Q, D, n, BH) || !make_map(&mk, K, D, m, BH) ||
+        !make_map(&mv, V, D, m, BH) || !make_map(&mdo, dO, D, n, BH) ||
+        !make_map_typed(&mdk, dK, D, m, BH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, 32) ||
+        !make_map_typed(&mdv, dV, D, m, BH, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, 32))
+        return ATTN_ERR_CUDA;
+    using CK = attn::kvtc::Cfg<D>;
+    using CQ = attn::dqtc::Cfg<D>;
+    auto kv = attn::kvtc::kv_kernel<D>;
+    auto dq = attn::dqtc::dq_kernel<D>;
+    if (cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, CK::kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, CQ::kSmemBytes) !=
+            cudaSuccess)
+        return ATTN_ERR_CUDA;
+    const int num_kt = (m + kTile - 1) / kTile, num_qt = (n + kTile - 1) / kTile;
+    const long long kv_items = static_cast<long long>(num_kt) * BH;
+    const long long dq_items = static_cast<long long>(num_qt) * BH;
+    if (kv_items > 0x7fffffffll || dq_items > 0x7fffffffll) return ATTN_ERR_SHAPE;
+    const int kv_grid = static_cast<int>(std::min<long long>(kv_items, sm_count()));
+    const int dq_grid = static_cast<int>(std::min<long long>(dq_items, sm_count()));
+    const int kv_hg = std::max(1, std::min(BH, 256 / num_kt));
+    const int dq_hg = std::max(1, std::min(BH, 256 / num_qt));
+    attn_status_t s = traced(ATTN_KERNEL_BWD_KV, st, [&] {
+        kv<<<static_cast<unsigned>(kv_grid), attn::kvtc::kThreads, CK::kSmemBytes, st>>>(
+            mq, mk, mv, mdo, mdk, mdv, lse2, Dd, counters + attn::bwdtc::kCntSched, n_pad, n, m, BH,
+            kv_hg, causal, scale, scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
+        return launched();
+    });
+    if (s != ATTN_OK) return s;
+    return traced(ATTN_KERNEL_BWD_DQ, st, [&] {
+        dq<<<static_cast<unsigned>(dq_grid), attn::dqtc::kThreads, CQ::kSmemBytes, st>>>(
+            mq, mk, mv, mdo, lse2, Dd, counters + attn::bwdtc::kCntSchedDq,
+            static_cast<__nv_bfloat16*>(dQ), n_pad, n, m, BH, dq_hg, causal, scale,
+            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
+        return launched();
+    });
+}
+
+// Which dQ design the bf16 tensor-core backward uses (ATTN_DQ_AUTO: the one
+// measured faster).
+bool dq_separate() {
+    return g_dq_path == ATTN_DQ_SEPARATE;
 }
 
 // fp32 by bf16 pieces: one CTA per (128-row tile, head), heads fastest.
@@ -475,7 +543,14 @@ extern "C" {
 attn_status_t attn_set_path(attn_path_t path) {
     if (path != ATTN_PATH_AUTO && path != ATTN_PATH_SIMT && path != ATTN_PATH_TENSOR)
         return ATTN_ERR_UNSUPPORTED;
-    g_path.store(path);
+    g_path = path;
+    return ATTN_OK;
+}
+
+attn_status_t attn_set_dq_path(attn_dq_path_t path) {
+    if (path != ATTN_DQ_AUTO && path != ATTN_DQ_REDUCE && path != ATTN_DQ_SEPARATE)
+        return ATTN_ERR_UNSUPPORTED;
+    g_dq_path = path;
     return ATTN_OK;
 }
 
@@ -550,28 +625,34 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const
     float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
     float* Dd = reinterpret_cast<float*>(ws + w.dd_off);
     float* dQacc = reinterpret_cast<float*>(ws + w.dq_off);
-    int* sched = reinterpret_cast<int*>(ws + w.sched_off);
+    int* counters = reinterpret_cast<int*>(ws + w.cnt_off);
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
 
-    // The tensor-core backwards take D already multiplied by the scale; the
-    // fp32 one writes dQ directly and needs no zeroed accumulator.
+    // The tensor-core backwards take D already multiplied by the scale. Only
+    // the paths that add dQ partials into the accumulator need it zeroed; the
+    // fp32 tensor-core backward and the separate dQ pass write dQ once.
     const float d_scale = tensor ? scale : 1.0f;
-    const bool zero_dq = path != Path::kTensorF32x;
+    const bool separate = path == Path::kTensorBf16 && dq_separate();
+    const bool zero_dq = path == Path::kSimt || (path == Path::kTensorBf16 && !separate);
     s = (dtype == ATTN_F32)
-            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv, d_scale,
-                                zero_dq, st)
-            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, sched, BH, n, w.n_pad, d, dv,
-                                        d_scale, zero_dq, st);
+            ? preprocess<float>(O, dO, LSE, lse2, Dd, dQacc, counters, w.n_counters, BH, n,
+                                w.n_pad, d, dv, d_scale, zero_dq, st)
+            : preprocess<__nv_bfloat16>(O, dO, LSE, lse2, Dd, dQacc, counters, w.n_counters, BH,
+                                        n, w.n_pad, d, dv, d_scale, zero_dq, st);
     if (s != ATTN_OK) return s;
     if (path == Path::kTensorF32x) {
         s = bwd_f32x(Q, K, V, dO, lse2, Dd, w.n_pad, dQ, dK, dV, BH, n, m, d, dv, causal, scale,
                      mask, st);
+    } else if (path == Path::kTensorBf16 && separate) {
+        s = (d == 64) ? bwd_separate<64>(Q, K, V, dO, lse2, Dd, counters, w.n_pad, dQ, dK, dV, BH,
+                                         n, m, causal, scale, mask, st)
+                      : bwd_separate<128>(Q, K, V, dO, lse2, Dd, counters, w.n_pad, dQ, dK, dV,
+                                          BH, n, m, causal, scale, mask, st);
     } else if (path == Path::kTensorBf16) {
-        s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
-                                       n, m, causal, scale, mask, st)
-                      : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, sched, w.n_pad, dQacc, dK, dV, BH,
-                                        n, m, causal, scale, mask, st);
-        if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, 1.0f, st);
+        s = (d == 64) ? bwd_tensor<64>(Q, K, V, dO, lse2, Dd, counters, w.n_pad, dQacc, dQ, dK,
+                                       dV, BH, n, m, causal, scale, mask, st)
+                      : bwd_tensor<128>(Q, K, V, dO, lse2, Dd, counters, w.n_pad, dQacc, dQ, dK,
+                                        dV, BH, n, m, causal, scale, mask, st);
     } else if (dtype == ATTN_F32) {
         s = bwd_simt<float>(Q, K, V, dO, LSE, Dd, w.n_pad, dQacc, dK, dV, BH, n, m, d, dv, causal,
                             scale, mask, st);
@@ -581,7 +662,7 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const
                                     causal, scale, mask, st);
         if (s == ATTN_OK) s = finalize<__nv_bfloat16>(dQacc, dQ, dq_elems, scale, st);
     }
-    if (s == ATTN_OK) g_last_launches = (path == Path::kTensorF32x) ? 2 : 3;
+    if (s == ATTN_OK) g_last_launches = (path == Path::kTensorF32x || (tensor && !separate)) ? 2 : 3;
     return s;
 }
 

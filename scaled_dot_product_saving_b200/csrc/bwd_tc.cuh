@@ -20,6 +20,17 @@
 // dV_j and dK_j stay in TMEM across all query tiles and are written once.
 // Folding `scale` into dS makes dK and dQ come out already scaled.
 //
+// dQ in bf16. Every key tile of a head adds a partial into the head's rows of
+// the fp32 accumulator (zeroed by the preprocess kernel). Once the partials of
+// a work item have landed, each warp of the dQ warpgroup counts the item in a
+// per-head counter in the workspace (a release add; nobody waits on it). Two
+// converter warps per CTA take 32-row slabs of dQ in head order from a global
+// counter, wait (polling with backoff) until every work item of the slab's
+// head has been counted, and convert the slab's finished sums to bf16 dQ. They
+// run beside the pipeline, so heads that finish early are converted while
+// later heads are still being computed, and at the end of the launch every
+// CTA helps with the last heads; no separate conversion pass runs.
+//
 // Two P/dS warpgroups split a tile into four chunks of 32 queries (two chunks
 // each) and signal each chunk as soon as its P^T/dS^T are in TMEM, so the MMA
 // thread issues that chunk's dV/dK k-steps while the chunks after it are
@@ -40,9 +51,10 @@
 // exact zeros ("Attention backward", Problem 8), so tiles wholly above the
 // diagonal are skipped.
 //
-// Warp roles (448 threads): warps 0-3 and 4-7 = the two P/dS warpgroups (TMEM
+// Warp roles (512 threads): warps 0-3 and 4-7 = the two P/dS warpgroups (TMEM
 // lane = key), warps 8-11 = dQ warpgroup (TMEM lane = query row), warp 12 =
-// TMA producer, warp 13 = TMEM allocator and MMA issuer.
+// TMA producer, warp 13 = TMEM allocator and MMA issuer, warps 14-15 = dQ
+// converters.
 //
 // TMEM (512 columns). d = 128: dV [0,128) dK [128,256) S^T [256,384)
 // dP^T [384,512); chunk c's P^T (bf16) goes to [256+32c, 256+32c+16) and its
@@ -62,10 +74,18 @@ namespace bwdtc {
 constexpr int kBN = 128;      // keys per work item
 constexpr int kBM = 128;      // queries per tile
 constexpr int kChunks = 4;    // 32-query chunks of a tile
-constexpr int kThreads = 448;
+constexpr int kThreads = 512;
 constexpr int kWarpDq = 8;         // first warp of the dQ warpgroup
 constexpr int kWarpProducer = 12;
 constexpr int kWarpMma = 13;
+constexpr int kWarpConv = 14;      // first of the two dQ converter warps
+constexpr int kConvWarps = 2;
+
+// Counters in the workspace (int32; all zeroed by the preprocess kernel).
+constexpr int kCntSched = 0;        // next work item
+constexpr int kCntConvClaim = 1;    // next dQ slab to convert
+constexpr int kCntSchedDq = 2;      // next work item of the separate dQ pass
+constexpr int kCntHeadBase = 64;    // [BH]: landed work items x 4 per head
 
 template <int D>
 struct Cfg {
@@ -197,15 +217,48 @@ __device__ __forceinline__ Item item_at(int b, int num_kt, int num_qt, int BH, i
     return it;
 }
 
+// The finished fp32 sums of one 32-row slab (rows row0.., clipped at n) of
+// head bh, read from the accumulator and written to dQ in bf16 by one warp:
+// D/4 lanes per row, 16 bytes each, sixteen rows' loads in flight per lane
+// group (D = 128: the whole slab in two rounds).
+template <int D>
+__device__ __forceinline__ void convert_slab(const float* acc, __nv_bfloat16* out, int bh, int row0,
+                                             int n, int lane) {
+    constexpr int kLanesPerRow = D / 4;
+    constexpr int kRowsPerIter = 32 / kLanesPerRow;
+    constexpr int kIters = 32 / kRowsPerIter;
+    constexpr int kBatch = kIters < 16 ? kIters : 16;
+    const int sub = lane / kLanesPerRow, c4 = (lane % kLanesPerRow) * 4;
+    const size_t base = size_t(bh) * n;
+#pragma unroll
+    for (int i0 = 0; i0 < kIters; i0 += kBatch) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int r = row0 + (i0 + u) * kRowsPerIter + sub;
+            v[u] = r < n ? __ldcg(reinterpret_cast<const float4*>(acc + (base + r) * D + c4))
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int r = row0 + (i0 + u) * kRowsPerIter + sub;
+            if (r < n)
+                *reinterpret_cast<uint2*>(out + (base + r) * D + c4) =
+                    make_uint2(pack_bf16x2(v[u].x, v[u].y), pack_bf16x2(v[u].z, v[u].w));
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
            const __grid_constant__ CUtensorMap tmdQacc, const __grid_constant__ CUtensorMap tmdK,
            const __grid_constant__ CUtensorMap tmdV, const float* __restrict__ lse2,
-           const float* __restrict__ Dd, int* __restrict__ sched, int n_pad, int n, int m, int BH,
-           int head_group, int causal, float scale, float scale_log2,
-           const int* __restrict__ key_len, int H, unsigned long long budget_ns) {
+           const float* __restrict__ Dd, int* __restrict__ counters, const float* dQacc,
+           __nv_bfloat16* __restrict__ dQ, int n_pad, int n, int m, int BH, int head_group,
+           int causal, float scale, float scale_log2, const int* __restrict__ key_len, int H,
+           unsigned long long budget_ns) {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Bars* bars = reinterpret_cast<Bars*>(smem + C::kOffBar);
@@ -357,7 +410,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // All of this item's loads are issued (a couple of tiles ahead of
             // the MMAs): take the next item now, publish it, and warm L2 with
             // its K/V.
-            int nb = G + atomicAdd(sched, 1);
+            int nb = G + atomicAdd(counters + kCntSched, 1);
             if (nb >= num_items) nb = -1;
             if (!publish(j + 1, nb)) { ok = false; break; }
             if (nb < 0) break;
@@ -711,11 +764,67 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 __syncwarp();
                 mbar_arrive(&bars->ds_smem_free);
             }
+            if (!ok) break;
+            // Every partial of this item has been handed to the TMA: once they
+            // have landed, count the item for its head (the converter warps
+            // wait for that count). The next item's first dQ is microseconds
+            // away (its K/V load and first tile come first), so this wait is
+            // off the pipeline's path.
+            if (lane == 0) {
+                bulk_wait_group0();
+                fence_proxy_async_global();
+                red_add_release_gpu(counters + kCntHeadBase + it.bh, 1);
+            }
+            __syncwarp();
         }
-        // The CTA may exit once the TMA has read its shared-memory sources;
-        // the reduce-adds themselves complete before the grid does.
-        if (lane == 0) bulk_wait_group_read0();
+        if (lane == 0) bulk_wait_group0();
         __syncwarp();
+        if (!ok) {
+            record_device_error(kErrTimeout);
+            *abort_flag = 1;
+        }
+    } else if (!aborted_early && warp >= kWarpConv && warp < kWarpConv + kConvWarps) {
+        // ------------------------------------------------ dQ converters
+        // Slabs of 32 rows, in head order (the order in which heads finish):
+        // claim one, wait until every work item of its head has landed its
+        // partials (4 counts per item, one per dQ warp), convert it.
+        const int num_qt = (n + kBM - 1) / kBM;
+        const int units = BH * num_qt * 4;
+        const int target = 4 * ((m + kBN - 1) / kBN);
+        bool ok = true;
+        for (;;) {
+            int u = 0;
+            if (lane == 0) u = atomicAdd(counters + kCntConvClaim, 1);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u >= units) break;
+            const int bh = u / (num_qt * 4);
+            const int row0 = (u % (num_qt * 4)) * 32;
+            // The wait gives up only if the count makes no progress for the
+            // time budget (a head of a long sequence legitimately takes long).
+            int ready = 1;
+            if (lane == 0) {
+                const int* cnt = counters + kCntHeadBase + bh;
+                uint64_t t0 = global_timer_ns();
+                uint32_t sleep_ns = 256;
+                int seen = -1;
+                for (int c; (c = ld_acquire_gpu(cnt)) < target;) {
+                    if (c != seen) {
+                        seen = c;
+                        t0 = global_timer_ns();
+                    } else if (*abort_flag || global_timer_ns() - t0 > budget_ns) {
+                        ready = 0;
+                        break;
+                    }
+                    __nanosleep(sleep_ns);
+                    if (sleep_ns < 4096) sleep_ns *= 2;
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ready, 0)) {
+                ok = false;
+                break;
+            }
+            if (row0 < n) convert_slab<D>(dQacc, dQ, bh, row0, n, lane);
+        }
         if (!ok) {
             record_device_error(kErrTimeout);
             *abort_flag = 1;

@@ -5,10 +5,13 @@
 //   O(n dv) instead of O(n m). It also writes the forward's LSE in base 2,
 //   and both arrays are padded to whole 128-row tiles (D = 0 and LSE = +inf
 //   in the padding, so padded query rows get P = 0 on the tensor-core path).
-//   The same launch zeroes the fp32 dQ accumulator and the tensor-core
-//   backward's work-item counter. D is stored multiplied by `d_scale` (the
-//   tensor-core backward folds the attention scale into it).
-// finalize: dQ = post_scale * dQacc, converted to the element type.
+//   The same launch zeroes the backward's counters (the tensor-core
+//   backward's work-item counter and its per-slab counts of landed dQ
+//   partials) and the fp32 dQ accumulator that the partials are added into.
+//   D is stored multiplied by `d_scale` (the tensor-core backward folds the
+//   attention scale into it).
+// finalize: dQ = post_scale * dQacc, converted to the element type (the
+//   CUDA-core backward only; the tensor-core backward writes dQ itself).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,27 +26,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Rows handled by groups of G = dv/8 lanes, 16-byte loads (bf16, dv % 8 == 0,
-// dv <= 256 so that G divides 32).
-__device__ __forceinline__ float row_dot_bf16_vec(const __nv_bfloat16* o, const __nv_bfloat16* g,
-                                                  int lane_in_group) {
-    const uint4 a = reinterpret_cast<const uint4*>(o)[lane_in_group];
-    const uint4 b = reinterpret_cast<const uint4*>(g)[lane_in_group];
-    float s = 0.f;
-    s = fmaf(bf16_lo(a.x), bf16_lo(b.x), s); s = fmaf(bf16_hi(a.x), bf16_hi(b.x), s);
-    s = fmaf(bf16_lo(a.y), bf16_lo(b.y), s); s = fmaf(bf16_hi(a.y), bf16_hi(b.y), s);
-    s = fmaf(bf16_lo(a.z), bf16_lo(b.z), s); s = fmaf(bf16_hi(a.z), bf16_hi(b.z), s);
-    s = fmaf(bf16_lo(a.w), bf16_lo(b.w), s); s = fmaf(bf16_hi(a.w), bf16_hi(b.w), s);
-    return s;
-}
+// Rows are handled by groups of G = dv/8 lanes with 16-byte loads (bf16,
+// dv % 8 == 0, dv <= 256 so that G divides 32).
+// Vectorised bf16 variant. Grid-stride over all BH * n_pad rows, kRowsInFlight
+// row groups per warp per step so that enough loads are in flight to cover
+// the memory latency.
+constexpr int kRowsInFlight = 4;
 
-// Vectorised bf16 variant. Grid-stride over all BH * n_pad rows.
 __global__ void __launch_bounds__(kThreads)
 preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                     const float* __restrict__ LSE, float* __restrict__ lse2,
-                    float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ sched,
-                    size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
+                    float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ counters,
+                    size_t n_counters, size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
+    for (size_t k = size_t(blockIdx.x) * kThreads + threadIdx.x; k < n_counters;
+         k += size_t(gridDim.x) * kThreads)
+        counters[k] = 0;
     const int G = dv / 8;                       // lanes per row
     const int rows_per_warp = 32 / G;
     const int lane = threadIdx.x & 31;
@@ -51,23 +48,42 @@ preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __
     const size_t warp_global = (size_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const size_t nwarps = (size_t(gridDim.x) * kThreads) >> 5;
     const size_t total_rows = size_t(BH) * n_pad;
-    for (size_t base = warp_global * rows_per_warp; base < total_rows;
-         base += nwarps * rows_per_warp) {
-        const size_t row = base + sub;
-        float s = 0.f;
-        bool real = false;
-        size_t src = 0;
-        if (row < total_rows) {
-            const size_t bh = row / n_pad;
-            const int i = int(row % n_pad);
-            real = i < n;
-            src = bh * size_t(n) + i;
-            if (real) s = row_dot_bf16_vec(O + src * dv, dO + src * dv, lig);
+    const size_t step_rows = size_t(rows_per_warp) * kRowsInFlight;
+    for (size_t base = warp_global * step_rows; base < total_rows; base += nwarps * step_rows) {
+        uint4 a[kRowsInFlight], b[kRowsInFlight];
+        float lse[kRowsInFlight];
+        bool real[kRowsInFlight];
+#pragma unroll
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            const size_t row = base + size_t(u) * rows_per_warp + sub;
+            real[u] = false;
+            a[u] = b[u] = make_uint4(0u, 0u, 0u, 0u);
+            lse[u] = 0.f;
+            if (row < total_rows) {
+                const size_t bh = row / n_pad;
+                const int i = int(row % n_pad);
+                if (i < n) {
+                    const size_t src = bh * size_t(n) + i;
+                    real[u] = true;
+                    a[u] = reinterpret_cast<const uint4*>(O + src * dv)[lig];
+                    b[u] = reinterpret_cast<const uint4*>(dO + src * dv)[lig];
+                    if (lig == 0) lse[u] = LSE[src];
+                }
+            }
         }
-        for (int off = G / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (row < total_rows && lig == 0) {
-            Dd[row] = real ? s * d_scale : 0.f;
-            lse2[row] = real ? LSE[src] * kLog2e : INFINITY;
+#pragma unroll
+        for (int u = 0; u < kRowsInFlight; ++u) {
+            const size_t row = base + size_t(u) * rows_per_warp + sub;
+            float sum = 0.f;
+            sum = fmaf(bf16_lo(a[u].x), bf16_lo(b[u].x), sum); sum = fmaf(bf16_hi(a[u].x), bf16_hi(b[u].x), sum);
+            sum = fmaf(bf16_lo(a[u].y), bf16_lo(b[u].y), sum); sum = fmaf(bf16_hi(a[u].y), bf16_hi(b[u].y), sum);
+            sum = fmaf(bf16_lo(a[u].z), bf16_lo(b[u].z), sum); sum = fmaf(bf16_hi(a[u].z), bf16_hi(b[u].z), sum);
+            sum = fmaf(bf16_lo(a[u].w), bf16_lo(b[u].w), sum); sum = fmaf(bf16_hi(a[u].w), bf16_hi(b[u].w), sum);
+            for (int off = G / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (row < total_rows && lig == 0) {
+                Dd[row] = real[u] ? sum * d_scale : 0.f;
+                lse2[row] = real[u] ? lse[u] * kLog2e : INFINITY;
+            }
         }
     }
     // zero the dQ accumulator (16-byte stores; dq_elems % 4 == 0)
@@ -86,9 +102,11 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 preprocess_generic(const T* __restrict__ O, const T* __restrict__ dO,
                    const float* __restrict__ LSE, float* __restrict__ lse2,
-                   float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ sched,
-                   size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) *sched = 0;
+                   float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ counters,
+                   size_t n_counters, size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
+    for (size_t k = size_t(blockIdx.x) * kThreads + threadIdx.x; k < n_counters;
+         k += size_t(gridDim.x) * kThreads)
+        counters[k] = 0;
     const int lane = threadIdx.x & 31;
     const size_t warp_global = (size_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const size_t nwarps = (size_t(gridDim.x) * kThreads) >> 5;

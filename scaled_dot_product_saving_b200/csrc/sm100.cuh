@@ -229,6 +229,26 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Order this thread's global accesses through the async proxy (TMA stores
+// and reduce-adds) against its generic-proxy accesses, in both directions.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------- inter-CTA counters (global)
+// Acquire load at GPU scope: later reads see what the releasing writers wrote
+// before their release.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Atomic add with release semantics at GPU scope and no result: this thread's
+// earlier writes are visible to whoever acquires the new value.
+__device__ __forceinline__ void red_add_release_gpu(int* p, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // --------------------------------------------------------------- tcgen05
 // TMEM allocation: executed by one whole warp; the base address is written
 // to shared memory.

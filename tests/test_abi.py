@@ -99,12 +99,36 @@ def test_tensor_path_request_rejects_other_shapes(L):
     assert L.lib.attn_set_path(9) == 4
 
 
+def test_path_setting_is_per_thread(L):
+    """attn_set_path in one host thread leaves the others' calls alone."""
+    import threading
+    seen = {}
+
+    def worker():
+        L.attn_set_path(L.ATTN_PATH_TENSOR)
+        seen["worker"] = fwd(L, d=32, dv=32)        # bf16 width 32: tensor path refuses
+    t = threading.Thread(target=worker)
+    t.start()
+    t.join()
+    assert seen["worker"] == 4
+    # This thread still has ATTN_PATH_AUTO: width 32 is accepted for the
+    # CUDA-core path and gets as far as the launch, which fails with no device.
+    if not torch.cuda.is_available():
+        assert fwd(L, d=32, dv=32) == 7
+    L.attn_set_path(L.ATTN_PATH_TENSOR)
+    try:
+        assert fwd(L, d=32, dv=32) == 4
+    finally:
+        L.attn_set_path(L.ATTN_PATH_AUTO)
+
+
 def test_workspace_size_formula(L):
     def expect(B, H, n, d):
         bh = B * H
         n_pad = -(-n // 128) * 128
         rows = -(-(bh * n_pad * 4) // 256) * 256
-        return 2 * rows + -(-(bh * n * d * 4) // 256) * 256 + 256
+        counters = 64 + bh                      # two counters padded to 256 bytes, then one per head
+        return 2 * rows + -(-(bh * n * d * 4) // 256) * 256 + -(-(counters * 4) // 256) * 256
     for (B, H, n, m, d) in [(1, 1, 1, 1, 1), (4, 16, 1024, 1024, 64), (2, 32, 4096, 4096, 128),
                             (8, 16, 512, 2048, 64), (1, 3, 77, 90, 40)]:
         assert L.attn_bwd_workspace_size(B, H, n, m, d, d, 1) == expect(B, H, n, d)

@@ -7,7 +7,7 @@ import pytest
 import torch
 
 import synth
-from parity_util import TOL, full_compare, heads_compare, gpu_run
+from parity_util import TOL, all_heads, full_compare, gpu_run, heads_compare
 
 pytestmark = pytest.mark.gpu
 
@@ -39,10 +39,14 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("dq_path", [lib.ATTN_DQ_REDUCE, lib.ATTN_DQ_SEPARATE],
+                         ids=["dq_reduce", "dq_separate"])
 @pytest.mark.parametrize("B,H,n,m,d,dv,dt,causal,lengths", CASES)
-def test_padding_mask(B, H, n, m, d, dv, dt, causal, lengths):
+def test_padding_mask(B, H, n, m, d, dv, dt, causal, lengths, dq_path):
+    if dq_path == lib.ATTN_DQ_SEPARATE and not (dt == "bf16" and d == dv and d in (64, 128)):
+        pytest.skip("the dQ design applies to the bf16 tensor-core path only")
     w = synth.make_small(B, H, n, m, d, dv, dt, causal, seed=B * 7 + n + m + d, lengths=lengths)
-    _assert_within(full_compare(w), TOL[dt], w.name)
+    _assert_within(full_compare(w, dq_path=dq_path), TOL[dt], w.name)
 
 
 def test_padded_rows_of_dk_dv_are_zero():
@@ -72,11 +76,12 @@ def test_lengths_out_of_range_are_clamped():
 
 def test_padded_full_size():
     """The padded workload at full size in the benchmark's launch
-    configuration: two complete heads, invariants over every head."""
+    configuration: every head element by element, and invariants."""
     w = synth.workload("padded_b8h16_n1024_d64")
-    errs, inv = heads_compare(w, [(0, 0), (3, 7), (w.B - 1, w.H - 1)])
-    _assert_within(errs, TOL["bf16"], w.name)
-    _assert_within(inv, TOL["bf16"], w.name + " invariants")
+    res = heads_compare(w, all_heads(w), dq_paths=(lib.ATTN_DQ_REDUCE, lib.ATTN_DQ_SEPARATE))
+    for p, (errs, inv) in res.items():
+        _assert_within(errs, TOL["bf16"], f"{w.name} dq path {p}")
+        _assert_within(inv, TOL["bf16"], f"{w.name} dq path {p} invariants")
 
 
 def test_no_mask_equals_full_length_mask():

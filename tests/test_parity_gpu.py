@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import synth
-from parity_util import TOL, full_compare, heads_compare
+from parity_util import TOL, all_heads, full_compare, heads_compare, scheduler_heads
 
 pytestmark = pytest.mark.gpu
 
@@ -15,8 +15,20 @@ lib = pytest.importorskip("scaled_dot_product_saving_b200")
 @pytest.fixture(autouse=True)
 def _auto_path():
     lib.attn_set_path(lib.ATTN_PATH_AUTO)
+    lib.attn_set_dq_path(lib.ATTN_DQ_AUTO)
     yield
     lib.attn_set_path(lib.ATTN_PATH_AUTO)
+    lib.attn_set_dq_path(lib.ATTN_DQ_AUTO)
+
+
+# The bf16 tensor-core backward's two dQ designs: partial sums reduce-added
+# into an accumulator, or a separate query-tile-major pass.
+DQ_PATHS = [lib.ATTN_DQ_REDUCE, lib.ATTN_DQ_SEPARATE]
+DQ_IDS = ["dq_reduce", "dq_separate"]
+
+
+def _tensor_bf16(dt, d, dv):
+    return dt == "bf16" and d == dv and d in (64, 128)
 
 
 def _assert_within(errs, tol, label):
@@ -55,10 +67,13 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("dq_path", DQ_PATHS, ids=DQ_IDS)
 @pytest.mark.parametrize("B,H,n,m,d,dv,dt,causal,std", SMALL)
-def test_small_shapes(B, H, n, m, d, dv, dt, causal, std):
+def test_small_shapes(B, H, n, m, d, dv, dt, causal, std, dq_path):
+    if dq_path == lib.ATTN_DQ_SEPARATE and not _tensor_bf16(dt, d, dv):
+        pytest.skip("the dQ design applies to the bf16 tensor-core path only")
     w = synth.make_small(B, H, n, m, d, dv, dt, causal, seed=B * 1000 + n + m + d, std_qk=std)
-    _assert_within(full_compare(w), TOL[dt], w.name)
+    _assert_within(full_compare(w, dq_path=dq_path), TOL[dt], w.name)
 
 
 @pytest.mark.parametrize("d,causal", [(64, True), (128, False)])
@@ -74,11 +89,12 @@ def test_cuda_core_path_bf16(d, causal):
     (4, 50, 300, 1000, 64, False),     # 400 / 1600 items, n != m, both ragged
     (1, 160, 130, 130, 128, True),     # one-key-tile items and one-tile pairs (has no tile B)
 ])
-def test_persistent_many_items(B, H, n, m, d, causal):
+@pytest.mark.parametrize("dq_path", DQ_PATHS, ids=DQ_IDS)
+def test_persistent_many_items(B, H, n, m, d, causal, dq_path):
     """Problems with more work items than SMs, so that every persistent CTA
     walks several items of different lengths (every head compared in full)."""
     w = synth.make_small(B, H, n, m, d, d, "bf16", causal, seed=B * H + n + d)
-    _assert_within(full_compare(w), TOL["bf16"], w.name)
+    _assert_within(full_compare(w, dq_path=dq_path), TOL["bf16"], w.name)
 
 
 @pytest.mark.parametrize("d,causal,scale", [
@@ -87,8 +103,10 @@ def test_persistent_many_items(B, H, n, m, d, causal):
     (128, False, 0.0),     # zero scale: uniform weights, dQ = dK = 0
     (64, True, 0.35),      # scale above 1/sqrt(d)
 ])
-def test_scale_values(d, causal, scale):
+@pytest.mark.parametrize("dq_path", DQ_PATHS, ids=DQ_IDS)
+def test_scale_values(d, causal, scale, dq_path):
     """Scales other than 1/sqrt(d) through the tensor-core path."""
+    lib.attn_set_dq_path(dq_path)
     import numpy as np
     import oracle.ref as ref
     from parity_util import rel_err, to64
@@ -110,29 +128,49 @@ def test_scale_values(d, causal, scale):
     _assert_within(errs, TOL["bf16"], f"d={d} causal={causal} scale={scale}")
 
 
-def test_tensor_path_is_taken():
+@pytest.mark.parametrize("dq_path,launches", [(lib.ATTN_DQ_REDUCE, 2), (lib.ATTN_DQ_SEPARATE, 3)],
+                         ids=DQ_IDS)
+def test_tensor_path_is_taken(dq_path, launches):
+    """preprocess + the fused backward (dQ written in it), or preprocess +
+    the dK/dV pass + the dQ pass."""
     lib.attn_set_path(lib.ATTN_PATH_TENSOR)
     w = synth.make_small(1, 1, 256, 256, 64, 64, "bf16", True, seed=3)
-    _assert_within(full_compare(w), TOL["bf16"], w.name)
-    assert lib.attn_last_launch_count() == 3
+    _assert_within(full_compare(w, dq_path=dq_path), TOL["bf16"], w.name)
+    assert lib.attn_last_launch_count() == launches      # of the backward call
 
 
 # ----------------------------------------------------------------------------
 # The four bf16 workloads at full size, in the launch configuration the
-# benchmark times: the first and last (batch, head) problems compared element
-# by element with the oracle, invariants checked over all heads.
+# benchmark times, compared element by element with the oracle head by head
+# (the worst head's error is kept), plus invariants over all heads:
+#  - the two small workloads: every head;
+#  - B2 H32 N4096: the first, middle and last head of every head group of the
+#    persistent schedules (groups of about 256 work items);
+#  - B1 H32 N16384: the groups there are two heads each; the first head of
+#    every group and the last head (a complete head of this size costs the
+#    float64 oracle several seconds).
 # ----------------------------------------------------------------------------
+def _full_size_heads(w):
+    if w.name in ("causal_b4h16_n1024_d64", "cross_b8h16_n512_m2048_d64"):
+        return all_heads(w)
+    if w.name == "causal_b1h32_n16384_d128":
+        return [(0, h) for h in range(0, w.H, 2)] + [(0, w.H - 1)]
+    return scheduler_heads(w)
+
+
 FULL = ["causal_b4h16_n1024_d64", "causal_b2h32_n4096_d128",
         "cross_b8h16_n512_m2048_d64", "causal_b1h32_n16384_d128"]
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_full_size(name):
+    """Both dQ designs, against one oracle evaluation per head."""
     w = synth.workload(name)
-    heads = [(0, 0), (w.B - 1, w.H - 1)]
-    errs, inv = heads_compare(w, heads)
-    _assert_within(errs, TOL["bf16"], name)
-    _assert_within(inv, TOL["bf16"], name + " invariants")
+    res = heads_compare(w, _full_size_heads(w), dq_paths=tuple(DQ_PATHS))
+    for p, label in zip(DQ_PATHS, DQ_IDS):
+        errs, inv = res[p]
+        _assert_within(errs, TOL["bf16"], f"{name} {label}")
+        _assert_within(inv, TOL["bf16"], f"{name} {label} invariants")
 
 
 def test_timeout_path_reports_error():

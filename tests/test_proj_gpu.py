@@ -68,7 +68,10 @@ def test_projection_backward_after_attention():
     want = ref.projection_backward(*(t.to(torch.float64).numpy() for t in (X, Wq, Wk, Wv)),
                                    dQr, dKr, dVr)
     errs = {name: rel_err(to64(g_), w) for name, g_, w in zip(("dX", "dWq", "dWk", "dWv"), got, want)}
-    assert all(v <= 3e-2 for v in errs.values()), errs
+    # The same 2e-2 bar: the chain rounds to bf16 twice (the attention
+    # gradients, then the projection outputs), which a CPU emulation of this
+    # arithmetic on these inputs puts at about 4e-3 of max|ref|.
+    assert all(v <= TOL["bf16"] for v in errs.values()), errs
 
 
 @pytest.mark.parametrize("B,n,d_model,H,dv", [
