@@ -103,10 +103,10 @@ attn_status_t attn_fwd(const void* Q, const void* K, const void* V,
  * attn_bwd_workspace_size -- bytes of device scratch that attn_bwd needs for
  * these sizes: D = rowsum(dO * O) and the LSE in base 2, both [B,H,n] fp32
  * padded to whole 128-row tiles, plus an fp32 [B,H,n,d] accumulator for dQ,
- * then 256 bytes for two counters of the persistent tensor-core backward
- * (its work items, and the dQ slabs its converter warps have claimed) and 4
- * bytes per (batch, head) for the head's count of finished work items (each
- * region rounded up to 256 bytes).
+ * then 256 bytes of counters of the persistent tensor-core backward (work
+ * items, and the dQ slabs its converter warps have claimed) and 4 bytes per
+ * (batch, head) for the head's count of finished work items (each region
+ * rounded up to 256 bytes).
  * Returns 0 if the sizes are invalid.
  */
 size_t attn_bwd_workspace_size(int B, int H, int n, int m, int d, int dv,

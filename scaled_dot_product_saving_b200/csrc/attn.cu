@@ -289,7 +289,7 @@ attn_status_t preprocess(const void* O, const void* dO, const float* LSE, float*
     if (vec) {
         const int rows_per_block =
             (attn::prep::kThreads / 32) * (32 / (dv / 8)) * attn::prep::kRowsInFlight;
-        const int grid = grid_for(rows, rows_per_block, sm_count() * 8);
+        const int grid = grid_for(rows, rows_per_block, sm_count() * attn::prep::kBlocksPerSm);
         return traced(ATTN_KERNEL_PREPROCESS, st, [&] {
             attn::prep::preprocess_bf16_vec<<<grid, attn::prep::kThreads, 0, st>>>(
                 static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), LSE,
@@ -362,11 +362,30 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     if (items > 0x7fffffffll) return ATTN_ERR_SHAPE;          // the kernel counts items in int
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     const int head_group = std::max(1, std::min(BH, 256 / num_kt));
+    // A programmatic dependent of the preprocess kernel launched just before
+    // it on the stream: its CTAs set up while the preprocess kernel finishes,
+    // and wait for its results in the kernel (griddepcontrol). Not while
+    // tracing: the early start would then be counted in this kernel's time.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(attn::bwdtc::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_trace.on ? 0 : 1;
+    __nv_bfloat16* dq16 = static_cast<__nv_bfloat16*>(dQ);
+    const float scale_log2 = scale * kLog2e;
+    const int* key_len = mask.key_len;
     return traced(ATTN_KERNEL_BWD_TENSOR, st, [&] {
-        kern<<<static_cast<unsigned>(grid), attn::bwdtc::kThreads, C::kSmemBytes, st>>>(
-            mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, counters, dQacc,
-            static_cast<__nv_bfloat16*>(dQ), n_pad, n, m, BH, head_group, causal, scale,
-            scale * kLog2e, mask.key_len, mask.H, kWaitBudgetNs);
+        if (cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mdo, mdq, mdk, mdv, lse2, Dd, counters, dQacc,
+                               dq16, n_pad, n, m, BH, head_group, causal, scale, scale_log2,
+                               key_len, mask.H, kWaitBudgetNs) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return ATTN_ERR_CUDA;
+        }
         return launched();
     });
 }
@@ -628,8 +647,8 @@ attn_status_t attn_bwd_masked(const void* Q, const void* K, const void* V, const
     int* counters = reinterpret_cast<int*>(ws + w.cnt_off);
     const size_t dq_elems = static_cast<size_t>(BH) * n * d;
 
-    // The tensor-core backwards take D already multiplied by the scale. Only
-    // the paths that add dQ partials into the accumulator need it zeroed; the
+    // The tensor-core backwards take D already multiplied by the scale. The
+    // paths that add dQ partials into the accumulator need it zeroed; the
     // fp32 tensor-core backward and the separate dQ pass write dQ once.
     const float d_scale = tensor ? scale : 1.0f;
     const bool separate = path == Path::kTensorBf16 && dq_separate();

@@ -25,11 +25,12 @@
 // a work item have landed, each warp of the dQ warpgroup counts the item in a
 // per-head counter in the workspace (a release add; nobody waits on it). Two
 // converter warps per CTA take 32-row slabs of dQ in head order from a global
-// counter, wait (polling with backoff) until every work item of the slab's
-// head has been counted, and convert the slab's finished sums to bf16 dQ. They
-// run beside the pipeline, so heads that finish early are converted while
-// later heads are still being computed, and at the end of the launch every
-// CTA helps with the last heads; no separate conversion pass runs.
+// claim counter, wait (polling with backoff) until every work item of the
+// slab's head has been counted, convert the slab's finished sums to bf16 dQ,
+// and drop the dead fp32 lines from L2 without writing them back. They run
+// beside the pipeline, so heads that finish early are converted while later
+// heads are still being computed, and at the end of the launch every CTA
+// helps with the last heads; no separate conversion pass runs.
 //
 // Two P/dS warpgroups split a tile into four chunks of 32 queries (two chunks
 // each) and signal each chunk as soon as its P^T/dS^T are in TMEM, so the MMA
@@ -87,15 +88,55 @@ constexpr int kCntConvClaim = 1;    // next dQ slab to convert
 constexpr int kCntSchedDq = 2;      // next work item of the separate dQ pass
 constexpr int kCntHeadBase = 64;    // [BH]: landed work items x 4 per head
 
+// Lane 0 of a warp: wait until *cnt reaches target. Gives up (false) on the
+// CTA's abort flag, or when the count has not moved for the time budget (a
+// count that keeps moving is a head still being worked on, however long).
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, const volatile int* abort,
+                                           uint64_t budget_ns) {
+    uint64_t t0 = global_timer_ns();
+    uint32_t sleep_ns = 128;
+    int seen = -1;
+    for (int c; (c = ld_acquire_gpu(cnt)) < target;) {
+        if (c != seen) {
+            seen = c;
+            t0 = global_timer_ns();
+        } else if (*abort || global_timer_ns() - t0 > budget_ns) {
+            return false;
+        }
+        __nanosleep(sleep_ns);
+        if (sleep_ns < 4096) sleep_ns *= 2;
+    }
+    return true;
+}
+
+// Drop one 32-row slab of the accumulator from L2 once converted: its sums
+// are dead, and the next call zeroes it again before use, so writing it back
+// to HBM would be wasted traffic. D/32 lines per row, one per lane and step.
+template <int D>
+__device__ __forceinline__ void discard_slab(const float* acc, int bh, int row0, int n, int lane) {
+    constexpr int kLinesPerRow = D / 32;
+    const size_t base = size_t(bh) * n;
+#pragma unroll
+    for (int i = 0; i < kLinesPerRow; ++i) {
+        const int idx = i * 32 + lane;
+        const int r = row0 + idx / kLinesPerRow;
+        if (r < n) discard_l2_line(acc + (base + r) * D + (idx % kLinesPerRow) * 32);
+    }
+}
+
 template <int D>
 struct Cfg {
-    static constexpr int kStages = (D == 64) ? 4 : 2;
+    // At d = 64 the K/V tiles are double-buffered (the next item's load runs
+    // during this item), with 3 Q/dO stages; d = 128 has room for neither.
+    static constexpr int kKV = (D == 64) ? 2 : 1;
+    static constexpr int kStages = (D == 64) ? 3 : 2;
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = 128 * D * 2;     // a 128-row bf16 tile
     static constexpr int kPanelBytes = 128 * 128;      // 128 rows x 128 B
-    static constexpr int kOffK = 0;
-    static constexpr int kOffV = kOffK + kTileBytes;
-    static constexpr int kOffQ = kOffV + kTileBytes;
+    static constexpr int kOffK = 0;                    // K/V buffer b: K at kOffK + b * kKVBytes,
+    static constexpr int kOffV = kOffK + kTileBytes;   // V kTileBytes after it
+    static constexpr int kKVBytes = 2 * kTileBytes;
+    static constexpr int kOffQ = kKV * kKVBytes;
     static constexpr int kOffdO = kOffQ + kStages * kTileBytes;
     static constexpr int kOffdS = kOffdO + kStages * kTileBytes;   // 128 keys x 128 queries
     static constexpr int kOffLse = kOffdS + 128 * 128 * 2;
@@ -118,8 +159,8 @@ struct Cfg {
 };
 
 struct Bars {
-    uint64_t kv_full;
-    uint64_t kv_empty;      // the item's last MMA has read K_j, V_j
+    uint64_t kv_full[2];
+    uint64_t kv_empty[2];   // the item's last MMA has read K_j, V_j of buffer b
     uint64_t q_full[4];
     uint64_t q_empty[4];
     uint64_t s_full;
@@ -302,8 +343,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const bool misaligned = (smem_addr(smem) & 1023u) != 0;
         if (misaligned) record_device_error(kErrTimeout);
         bars->abort = (misaligned || *reinterpret_cast<volatile unsigned int*>(&g_device_error) != 0) ? 1 : 0;
-        mbar_init(&bars->kv_full, 1);
-        mbar_init(&bars->kv_empty, 1);
+        for (int kb = 0; kb < 2; ++kb) {
+            mbar_init(&bars->kv_full[kb], 1);
+            mbar_init(&bars->kv_empty[kb], 1);
+        }
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
@@ -333,6 +376,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const bool aborted_early = bars->abort != 0;
+    // Launched as a programmatic dependent of the preprocess kernel: the
+    // setup above overlapped its tail; its outputs (LSE_2, D, the zeroed
+    // accumulator and counters) are touched only after this.
+    grid_dependency_wait();
 
     if (!aborted_early && warp == kWarpProducer && lane == 0) {
         // ------------------------------------------------ TMA producer
@@ -392,14 +439,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             // V_j once the previous item's last MMA has read its own.
             if (!load_q(it, 0, g)) { ok = false; break; }
             ++g;
-            if (j > 0 && !mbar_wait(&bars->kv_empty, (j - 1) & 1, abort_flag, budget_ns)) {
+            const int kb = j % C::kKV;
+            if (j >= C::kKV &&
+                !mbar_wait(&bars->kv_empty[kb], (j / C::kKV - 1) & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
-            mbar_arrive_expect_tx(&bars->kv_full, 2 * C::kTileBytes);
+            mbar_arrive_expect_tx(&bars->kv_full[kb], 2 * C::kTileBytes);
             for (int p = 0; p < C::kPanels; ++p) {
-                tma_load_3d(smem + C::kOffK + p * C::kPanelBytes, &tmK, &bars->kv_full, p * 64, it.k0, it.bh);
-                tma_load_3d(smem + C::kOffV + p * C::kPanelBytes, &tmV, &bars->kv_full, p * 64, it.k0, it.bh);
+                tma_load_3d(smem + C::kOffK + kb * C::kKVBytes + p * C::kPanelBytes, &tmK,
+                            &bars->kv_full[kb], p * 64, it.k0, it.bh);
+                tma_load_3d(smem + C::kOffV + kb * C::kKVBytes + p * C::kPanelBytes, &tmV,
+                            &bars->kv_full[kb], p * 64, it.k0, it.bh);
             }
             ++kv_issued;
             for (int t = 1; t < it.T; ++t) {
@@ -426,9 +477,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             *abort_flag = 1;
         }
         // Drain: every load issued must land before the CTA may exit. Loads
-        // older than the last stage's worth (and K/V before the last) were
-        // consumed, so they have landed.
-        if (kv_issued > 0) (void)mbar_wait_timed(&bars->kv_full, (kv_issued - 1) & 1, budget_ns);
+        // older than the last stage's worth (and K/V before the last buffer's
+        // worth) were consumed, so they have landed.
+        for (int i = (kv_issued > C::kKV ? kv_issued - C::kKV : 0); i < kv_issued; ++i)
+            (void)mbar_wait_timed(&bars->kv_full[i % C::kKV], (i / C::kKV) & 1, budget_ns);
         for (int t = (g > C::kStages ? g - C::kStages : 0); t < g; ++t)
             (void)mbar_wait_timed(&bars->q_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
     } else if (!aborted_early && warp == kWarpMma && lane == 0) {
@@ -436,8 +488,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
         constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 1, 1);      // dQ
-        const uint32_t sK = smem_addr(smem + C::kOffK);
-        const uint32_t sV = smem_addr(smem + C::kOffV);
+        uint32_t sK = smem_addr(smem + C::kOffK), sV = smem_addr(smem + C::kOffV);   // per item
         const uint32_t sdS = smem_addr(smem + C::kOffdS);
         // dP^T(g) = V dO(g)^T once Q/dO(g) are in; its columns are free once
         // the previous tile's dK MMAs (issued earlier) have read dS^T.
@@ -479,10 +530,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const int T = item(b).T;
-            if (!mbar_wait(&bars->kv_full, j & 1, abort_flag, budget_ns)) {
+            const int kb = j % C::kKV;
+            if (!mbar_wait(&bars->kv_full[kb], (j / C::kKV) & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
+            sK = smem_addr(smem + C::kOffK + kb * C::kKVBytes);
+            sV = smem_addr(smem + C::kOffV + kb * C::kKVBytes);
             // At d = 64 (dQ in columns of its own) the next tile's dP^T and S^T
             // are issued right after this tile's dV/dK MMAs, before the dQ MMA
             // waits for the dS tile, so the P/dS warps start on tile t+1 while
@@ -552,7 +606,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 mma_commit(&bars->dq_full);
                 // The item's last MMA has been issued: K_j, V_j are free once
                 // it has completed.
-                if (t == T - 1) mma_commit(&bars->kv_empty);
+                if (t == T - 1) mma_commit(&bars->kv_empty[kb]);
             }
         }
         if (!ok) {
@@ -785,45 +839,31 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
     } else if (!aborted_early && warp >= kWarpConv && warp < kWarpConv + kConvWarps) {
         // ------------------------------------------------ dQ converters
-        // Slabs of 32 rows, in head order (the order in which heads finish):
-        // claim one, wait until every work item of its head has landed its
-        // partials (4 counts per item, one per dQ warp), convert it.
-        const int num_qt = (n + kBM - 1) / kBM;
+        // Slabs of 32 rows, in head order (the order in which heads finish).
         const int units = BH * num_qt * 4;
-        const int target = 4 * ((m + kBN - 1) / kBN);
+        const int target = 4 * num_kt;
         bool ok = true;
-        for (;;) {
+        // Conversion: claim a slab, wait until every work item of its head
+        // has landed its partials (4 counts per item, one per dQ warp),
+        // convert it, drop its fp32 lines.
+        for (; ok;) {
             int u = 0;
             if (lane == 0) u = atomicAdd(counters + kCntConvClaim, 1);
             u = __shfl_sync(0xffffffffu, u, 0);
             if (u >= units) break;
             const int bh = u / (num_qt * 4);
             const int row0 = (u % (num_qt * 4)) * 32;
-            // The wait gives up only if the count makes no progress for the
-            // time budget (a head of a long sequence legitimately takes long).
             int ready = 1;
-            if (lane == 0) {
-                const int* cnt = counters + kCntHeadBase + bh;
-                uint64_t t0 = global_timer_ns();
-                uint32_t sleep_ns = 256;
-                int seen = -1;
-                for (int c; (c = ld_acquire_gpu(cnt)) < target;) {
-                    if (c != seen) {
-                        seen = c;
-                        t0 = global_timer_ns();
-                    } else if (*abort_flag || global_timer_ns() - t0 > budget_ns) {
-                        ready = 0;
-                        break;
-                    }
-                    __nanosleep(sleep_ns);
-                    if (sleep_ns < 4096) sleep_ns *= 2;
-                }
-            }
+            if (lane == 0) ready = wait_count(counters + kCntHeadBase + bh, target, abort_flag, budget_ns);
             if (!__shfl_sync(0xffffffffu, ready, 0)) {
                 ok = false;
                 break;
             }
-            if (row0 < n) convert_slab<D>(dQacc, dQ, bh, row0, n, lane);
+            if (row0 < n) {
+                convert_slab<D>(dQacc, dQ, bh, row0, n, lane);
+                __syncwarp();
+                discard_slab<D>(dQacc, bh, row0, n, lane);
+            }
         }
         if (!ok) {
             record_device_error(kErrTimeout);

@@ -5,17 +5,18 @@
 //   O(n dv) instead of O(n m). It also writes the forward's LSE in base 2,
 //   and both arrays are padded to whole 128-row tiles (D = 0 and LSE = +inf
 //   in the padding, so padded query rows get P = 0 on the tensor-core path).
-//   The same launch zeroes the backward's counters (the tensor-core
-//   backward's work-item counter and its per-slab counts of landed dQ
-//   partials) and the fp32 dQ accumulator that the partials are added into.
-//   D is stored multiplied by `d_scale` (the tensor-core backward folds the
-//   attention scale into it).
+//   The same launch zeroes the backwards' counters (work items, claims and
+//   per-head counts) and, for the backwards that add dQ partials into the
+//   fp32 accumulator, the accumulator. D is stored multiplied by `d_scale`
+//   (the tensor-core backward folds the attention scale into it).
 // finalize: dQ = post_scale * dQacc, converted to the element type (the
 //   CUDA-core backward only; the tensor-core backward writes dQ itself).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
+
+#include "sm100.cuh"
 
 namespace attn {
 namespace prep {
@@ -30,14 +31,18 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 // dv % 8 == 0, dv <= 256 so that G divides 32).
 // Vectorised bf16 variant. Grid-stride over all BH * n_pad rows, kRowsInFlight
 // row groups per warp per step so that enough loads are in flight to cover
-// the memory latency.
+// the memory latency. The grid is one wave (kBlocksPerSm per SM): no later
+// wave competes for SMs with the backward's CTAs, which start under this
+// kernel's tail.
 constexpr int kRowsInFlight = 4;
+constexpr int kBlocksPerSm = 3;
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kBlocksPerSm)
 preprocess_bf16_vec(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                     const float* __restrict__ LSE, float* __restrict__ lse2,
                     float* __restrict__ Dd, float* __restrict__ dQacc, int* __restrict__ counters,
                     size_t n_counters, size_t dq_elems, int BH, int n, int n_pad, int dv, float d_scale) {
+    grid_launch_dependents();           // the backward may start its prologue
     for (size_t k = size_t(blockIdx.x) * kThreads + threadIdx.x; k < n_counters;
          k += size_t(gridDim.x) * kThreads)
         counters[k] = 0;

@@ -235,6 +235,19 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// ------------------------------------------ programmatic dependent launch
+// Let the next kernel in the stream, if launched as a programmatic dependent,
+// start its prologue now (it still waits for this grid's results, below).
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grid this one depends on (the previous kernel in the stream,
+// when launched as a programmatic dependent) has completed and its writes are
+// visible; returns at once otherwise.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------- inter-CTA counters (global)
 // Acquire load at GPU scope: later reads see what the releasing writers wrote
 // before their release.
@@ -242,6 +255,11 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
+}
+// Drop the 128-byte L2 line holding `p` without writing it back (its data
+// becomes undefined): for scratch whose contents are dead.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 // Atomic add with release semantics at GPU scope and no result: this thread's
 // earlier writes are visible to whoever acquires the new value.

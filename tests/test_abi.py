@@ -127,7 +127,7 @@ def test_workspace_size_formula(L):
         bh = B * H
         n_pad = -(-n // 128) * 128
         rows = -(-(bh * n_pad * 4) // 256) * 256
-        counters = 64 + bh                      # two counters padded to 256 bytes, then one per head
+        counters = 64 + bh                      # counters padded to 256 bytes, then one per head
         return 2 * rows + -(-(bh * n * d * 4) // 256) * 256 + -(-(counters * 4) // 256) * 256
     for (B, H, n, m, d) in [(1, 1, 1, 1, 1), (4, 16, 1024, 1024, 64), (2, 32, 4096, 4096, 128),
                             (8, 16, 512, 2048, 64), (1, 3, 77, 90, 40)]:
