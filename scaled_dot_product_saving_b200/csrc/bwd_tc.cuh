@@ -192,24 +192,28 @@ __device__ __forceinline__ void pds_half(int q0, const uint32_t (&sr)[16], const
                                          int keys_masked_below, float scale, float scale_log2,
                                          uint32_t pcol, uint32_t dscol, uint32_t* dk) {
     uint32_t pk[8];
+    // Pairs of queries through the paired fp32 instructions (each half
+    // rounded exactly as the scalar one), which halve the FMA-pipe issue.
+    const f32x2 sl2 = make_f32x2(scale_log2, scale_log2), sc2 = make_f32x2(scale, scale);
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q0 + 4 * g);
         const float4 d4 = *reinterpret_cast<const float4*>(dd_s + q0 + 4 * g);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-        float p[4], ds[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            const int e = 4 * g + h;
-            p[h] = ex2(fmaf(__uint_as_float(sr[e]), scale_log2, -lv[h]));
-            if (MASKED && (q0 + e) < keys_masked_below) p[h] = 0.f;
-            ds[h] = p[h] * fmaf(__uint_as_float(pr[e]), scale, -dv[h]);
+        for (int h = 0; h < 2; ++h) {
+            const int e = 4 * g + 2 * h;
+            const float2 x = split_f32x2(fma_x2(
+                make_f32x2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sl2,
+                h ? make_f32x2(-l4.z, -l4.w) : make_f32x2(-l4.x, -l4.y)));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
+            if (MASKED && (q0 + e) < keys_masked_below) p0 = 0.f;
+            if (MASKED && (q0 + e + 1) < keys_masked_below) p1 = 0.f;
+            const f32x2 t = fma_x2(make_f32x2(__uint_as_float(pr[e]), __uint_as_float(pr[e + 1])), sc2,
+                                   h ? make_f32x2(-d4.z, -d4.w) : make_f32x2(-d4.x, -d4.y));
+            const float2 ds = split_f32x2(mul_x2(make_f32x2(p0, p1), t));
+            pk[2 * g + h] = pack_bf16x2(p0, p1);
+            dk[2 * g + h] = pack_bf16x2(ds.x, ds.y);
         }
-        pk[2 * g] = pack_bf16x2(p[0], p[1]);
-        pk[2 * g + 1] = pack_bf16x2(p[2], p[3]);
-        dk[2 * g] = pack_bf16x2(ds[0], ds[1]);
-        dk[2 * g + 1] = pack_bf16x2(ds[2], ds[3]);
     }
     tmem_st8(pcol, pk);
     tmem_st8(dscol, dk);

@@ -122,6 +122,15 @@ def test_path_setting_is_per_thread(L):
         L.attn_set_path(L.ATTN_PATH_AUTO)
 
 
+def test_dq_path_setting(L):
+    """attn_set_dq_path takes the three designs and refuses other values."""
+    for p in (L.ATTN_DQ_REDUCE, L.ATTN_DQ_SEPARATE, L.ATTN_DQ_AUTO):
+        assert L.lib.attn_set_dq_path(p) == 0
+    assert L.lib.attn_set_dq_path(7) == 4
+    assert L.lib.attn_set_dq_path(-1) == 4
+    L.attn_set_dq_path(L.ATTN_DQ_AUTO)
+
+
 def test_workspace_size_formula(L):
     def expect(B, H, n, d):
         bh = B * H
