@@ -785,37 +785,45 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     break;
                 }
                 tc_fence_after();
-                // 64 columns at a time; the TMEM columns are released (dq_free)
-                // as soon as the last of them is in registers.
+                // 32 columns (one segment) at a time through two register
+                // buffers: segment sg + 2 is loaded from TMEM as soon as
+                // segment sg has been written to shared memory, so the loads
+                // overlap the staging and the TMEM columns are released
+                // (dq_free) as soon as the last segment is in registers.
+                constexpr int kSegs = D / 32;
+                uint32_t va[32], vb[32];
+                tmem_ld32(tl + C::kColdQ, va);
+                tmem_ld32(tl + C::kColdQ + 32, vb);
+                tmem_ld_wait();
+                if (kSegs == 2) {
+                    tc_fence_before();
+                    mbar_arrive(&bars->dq_free);
+                }
 #pragma unroll
-                for (int pair = 0; pair < D / 64; ++pair) {
-                    uint32_t v[64];
-                    tmem_ld32(tl + C::kColdQ + 64 * pair, *reinterpret_cast<uint32_t(*)[32]>(v));
-                    tmem_ld32(tl + C::kColdQ + 64 * pair + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                    tmem_ld_wait();
-                    if (pair == D / 64 - 1) {
-                        tc_fence_before();
-                        mbar_arrive(&bars->dq_free);
+                for (int sg = 0; sg < kSegs; ++sg) {                  // columns 32sg..32sg+31
+                    uint32_t (&v)[32] = (sg & 1) ? vb : va;
+                    uint8_t* buf = stage + (sg & 1) * 4096;
+                    if (sg >= 2) {
+                        if (lane == 0) bulk_wait_group_read1();       // buffer's previous segment read
+                        __syncwarp();
                     }
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int sg = 2 * pair + hh;                 // columns 32sg..32sg+31
-                        uint8_t* buf = stage + hh * 4096;
-                        if (sg >= 2) {
-                            if (lane == 0) bulk_wait_group_read1();   // buffer's previous segment read
-                            __syncwarp();
+                    for (int k = 0; k < 8; ++k)
+                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
+                            make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                    if (sg + 2 < kSegs) {
+                        tmem_ld32(tl + C::kColdQ + 32 * (sg + 2), v);
+                        if (sg + 3 == kSegs) {
+                            tmem_ld_wait();
+                            tc_fence_before();
+                            mbar_arrive(&bars->dq_free);
                         }
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((k ^ (lane & 7)) * 16)) =
-                                make_uint4(v[32 * hh + 4 * k], v[32 * hh + 4 * k + 1],
-                                           v[32 * hh + 4 * k + 2], v[32 * hh + 4 * k + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_reduce_add_3d(&tmdQacc, buf, 32 * sg, row0, it.bh);
-                            bulk_commit_group();
-                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_reduce_add_3d(&tmdQacc, buf, 32 * sg, row0, it.bh);
+                        bulk_commit_group();
                     }
                 }
                 if (lane == 0) bulk_wait_group_read0();
