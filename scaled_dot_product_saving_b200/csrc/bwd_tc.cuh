@@ -29,8 +29,9 @@
 // slab's head has been counted, convert the slab's finished sums to bf16 dQ,
 // and drop the dead fp32 lines from L2 without writing them back. They run
 // beside the pipeline, so heads that finish early are converted while later
-// heads are still being computed, and at the end of the launch every CTA
-// helps with the last heads; no separate conversion pass runs.
+// heads are still being computed; every other warp of a CTA joins them once
+// its own work has run out, so the last heads, which finish together, are
+// converted by all warps of all CTAs. No separate conversion pass runs.
 //
 // Two P/dS warpgroups split a tile into four chunks of 32 queries (two chunks
 // each) and signal each chunk as soon as its P^T/dS^T are in TMEM, so the MMA
@@ -104,7 +105,7 @@ __device__ __forceinline__ bool wait_count(const int* cnt, int target, const vol
             return false;
         }
         __nanosleep(sleep_ns);
-        if (sleep_ns < 4096) sleep_ns *= 2;
+        if (sleep_ns < 1024) sleep_ns *= 2;
     }
     return true;
 }
@@ -234,13 +235,27 @@ __device__ __forceinline__ void store_ds_chunk(uint8_t* sdS, int c, int r, const
 }
 
 // The (head, key tile) of work item `b` in schedule order (see the kernel's
-// comment).
-__device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int& bh, int& kt) {
-    const int group = b / (hg * num_kt);
-    const int within = b % (hg * num_kt);
-    const int heads_here = min(hg, BH - group * hg);
+// comment). When causal, the last two groups form one: a group's longest
+// items run about as long as the whole group takes on all SMs, so in a last
+// group of the usual size they would end well after every other CTA.
+__device__ __forceinline__ void cta_tile(int b, int num_kt, int BH, int hg, int causal, int& bh,
+                                         int& kt) {
+    const int groups = (BH + hg - 1) / hg;
+    const int tail_groups = causal ? 2 : 1;
+    const int tail_head = groups >= tail_groups ? (groups - tail_groups) * hg : 0;   // last group's first head
+    const int tail_item = tail_head * num_kt;
+    int head0, heads_here, within;
+    if (b < tail_item) {
+        head0 = (b / (hg * num_kt)) * hg;
+        heads_here = hg;
+        within = b % (hg * num_kt);
+    } else {
+        head0 = tail_head;
+        heads_here = BH - tail_head;
+        within = b - tail_item;
+    }
     kt = within / heads_here;
-    bh = group * hg + within % heads_here;
+    bh = head0 + within % heads_here;
 }
 
 // One work item: 128 keys of one head and the query tiles that see them.
@@ -254,7 +269,7 @@ __device__ __forceinline__ Item item_at(int b, int num_kt, int num_qt, int BH, i
                                         const int* key_len, int H, int m) {
     Item it;
     int kt;
-    cta_tile(b, num_kt, BH, hg, it.bh, kt);
+    cta_tile(b, num_kt, BH, hg, causal, it.bh, kt);
     it.k0 = kt * kBN;
     it.mk = keys_valid(key_len, it.bh, H, m);
     it.first_qt = causal ? kt : 0;
@@ -385,6 +400,37 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     // accumulator and counters) are touched only after this.
     grid_dependency_wait();
 
+    // dQ conversion, by one warp: slabs of 32 rows in head order (the order in
+    // which heads finish). Claim a slab, wait until every work item of its
+    // head has landed its partials (4 counts per item, one per dQ warp),
+    // convert it, drop its fp32 lines; until no slab is left.
+    auto convert_loop = [&]() {
+        const int units = BH * num_qt * 4;
+        const int target = 4 * num_kt;
+        for (;;) {
+            int u = 0;
+            if (lane == 0) u = atomicAdd(counters + kCntConvClaim, 1);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u >= units) return;
+            const int bh = u / (num_qt * 4);
+            const int row0 = (u % (num_qt * 4)) * 32;
+            int ready = 1;
+            if (lane == 0) ready = wait_count(counters + kCntHeadBase + bh, target, abort_flag, budget_ns);
+            if (!__shfl_sync(0xffffffffu, ready, 0)) {
+                if (lane == 0) {
+                    record_device_error(kErrTimeout);
+                    *abort_flag = 1;
+                }
+                return;
+            }
+            if (row0 < n) {
+                convert_slab<D>(dQacc, dQ, bh, row0, n, lane);
+                __syncwarp();
+                discard_slab<D>(dQacc, bh, row0, n, lane);
+            }
+        }
+    };
+
     if (!aborted_early && warp == kWarpProducer && lane == 0) {
         // ------------------------------------------------ TMA producer
         prefetch_tensor_map(&tmQ);
@@ -487,8 +533,11 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             (void)mbar_wait_timed(&bars->kv_full[i % C::kKV], (i / C::kKV) & 1, budget_ns);
         for (int t = (g > C::kStages ? g - C::kStages : 0); t < g; ++t)
             (void)mbar_wait_timed(&bars->q_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
+    } else if (!aborted_early && warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
+        // The whole warp walks the loop (waits are warp-wide) and one elected
+        // lane issues the MMAs and commits.
+        const uint32_t leader = elect_leader();
         constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
         constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 1, 1);      // dQ
@@ -498,14 +547,14 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // the previous tile's dK MMAs (issued earlier) have read dS^T.
         auto issue_dP = [&](int g) -> bool {
             const int s = g % C::kStages;
-            if (!mbar_wait(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
+            if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
             tc_fence_after();
             const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
+                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                         sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0, leader);
             }
             return true;
         };
@@ -514,28 +563,28 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // warpgroup has read it out.
         auto issue_S = [&](int g) -> bool {
             if (C::kAlias && g > 0 &&
-                !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns))
+                !mbar_wait_warp(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns))
                 return false;
             tc_fence_after();
             const uint32_t sQ = smem_addr(smem + C::kOffQ + (g % C::kStages) * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
-                       sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
+                mma_ss_w(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
+                         sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0, leader);
             }
-            mma_commit(&bars->s_full);
+            mma_commit_w(&bars->s_full, leader);
             return true;
         };
         bool ok = true;
         int g = 0;
         for (int j = 0; ok; ++j) {
-            const int b = next_item(j, false);
+            const int b = next_item(j, true);
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const int T = item(b).T;
             const int kb = j % C::kKV;
-            if (!mbar_wait(&bars->kv_full[kb], (j / C::kKV) & 1, abort_flag, budget_ns)) {
+            if (!mbar_wait_warp(&bars->kv_full[kb], (j / C::kKV) & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
@@ -558,7 +607,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 // The item's first dV/dK MMAs overwrite the accumulators: the
                 // previous item's epilogue must have read them out.
                 if (t == 0 && j > 0 &&
-                    !mbar_wait(&bars->acc_free, (j - 1) & 1, abort_flag, budget_ns)) {
+                    !mbar_wait_warp(&bars->acc_free, (j - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -568,7 +617,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 bool first = (t == 0);
                 for (int ci = 0; ci < kChunks; ++ci) {
                     const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
-                    if (!mbar_wait(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -576,16 +625,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
-                        mma_ts(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
-                               sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
-                        mma_ts(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
-                               sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                        mma_ts_w(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
+                                 sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
+                        mma_ts_w(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
+                                 sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&bars->q_empty[s]);
-                if (t == T - 1) mma_commit(&bars->acc_done);
+                mma_commit_w(&bars->q_empty[s], leader);
+                if (t == T - 1) mma_commit_w(&bars->acc_done, leader);
                 if (!C::kAlias && t + 1 < T) {
                     if (!issue_dP(g + 1) || !issue_S(g + 1)) {
                         ok = false;
@@ -594,30 +643,30 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     ahead = true;
                 }
                 if (!C::kAlias && g > 0 &&
-                    !mbar_wait(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
+                    !mbar_wait_warp(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
-                if (!mbar_wait(&bars->ds_smem_full, g & 1, abort_flag, budget_ns)) {
+                if (!mbar_wait_warp(&bars->ds_smem_full, g & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ss(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
-                           sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0);
-                mma_commit(&bars->dq_full);
+                    mma_ss_w(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
+                             sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0, leader);
+                mma_commit_w(&bars->dq_full, leader);
                 // The item's last MMA has been issued: K_j, V_j are free once
                 // it has completed.
-                if (t == T - 1) mma_commit(&bars->kv_empty[kb]);
+                if (t == T - 1) mma_commit_w(&bars->kv_empty[kb], leader);
             }
         }
         if (!ok) {
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
-        mma_commit(&bars->mma_drain);
+        mma_commit_w(&bars->mma_drain, leader);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
     } else if (!aborted_early && warp < 8) {
         // ------------------------------------------------ P / dS warpgroups
@@ -851,37 +900,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
     } else if (!aborted_early && warp >= kWarpConv && warp < kWarpConv + kConvWarps) {
         // ------------------------------------------------ dQ converters
-        // Slabs of 32 rows, in head order (the order in which heads finish).
-        const int units = BH * num_qt * 4;
-        const int target = 4 * num_kt;
-        bool ok = true;
-        // Conversion: claim a slab, wait until every work item of its head
-        // has landed its partials (4 counts per item, one per dQ warp),
-        // convert it, drop its fp32 lines.
-        for (; ok;) {
-            int u = 0;
-            if (lane == 0) u = atomicAdd(counters + kCntConvClaim, 1);
-            u = __shfl_sync(0xffffffffu, u, 0);
-            if (u >= units) break;
-            const int bh = u / (num_qt * 4);
-            const int row0 = (u % (num_qt * 4)) * 32;
-            int ready = 1;
-            if (lane == 0) ready = wait_count(counters + kCntHeadBase + bh, target, abort_flag, budget_ns);
-            if (!__shfl_sync(0xffffffffu, ready, 0)) {
-                ok = false;
-                break;
-            }
-            if (row0 < n) {
-                convert_slab<D>(dQacc, dQ, bh, row0, n, lane);
-                __syncwarp();
-                discard_slab<D>(dQacc, bh, row0, n, lane);
-            }
-        }
-        if (!ok) {
-            record_device_error(kErrTimeout);
-            *abort_flag = 1;
-        }
+        convert_loop();
     }
+    // A warp whose own work has run out helps with the conversion: at the end
+    // of the launch the last heads finish together, and two warps per CTA
+    // would take several rounds of slabs for them.
+    __syncwarp();
+    if (!aborted_early && warp < kWarpConv && *abort_flag == 0) convert_loop();
 
     tc_fence_before();
     __syncthreads();

@@ -295,8 +295,11 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             (void)mbar_wait_timed(&bars->k_full[t % C::kKStages], (t / C::kKStages) & 1, budget_ns);
         for (int t = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); t < v_issued; ++t)
             (void)mbar_wait_timed(&bars->v_full[t % C::kVStages], (t / C::kVStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
+    } else if (!aborted_early && warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
+        // The whole warp walks the loop (waits are warp-wide) and one elected
+        // lane issues the MMAs and commits.
+        const uint32_t leader = elect_leader();
         constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, 0, 0);   // S, dP
         constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 0, 1);     // dQ (B = K_j MN-major)
         const uint32_t sQ = smem_addr(smem + C::kOffQ);
@@ -306,31 +309,31 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColS0 + 128 * (c & 1), sdesc_sw128(sQ + koff, 16, 1024),
-                       sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0);
+                mma_ss_w(tmem + C::kColS0 + 128 * (c & 1), sdesc_sw128(sQ + koff, 16, 1024),
+                         sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0, leader);
             }
-            mma_commit(&bars->s_full[c & 1]);
+            mma_commit_w(&bars->s_full[c & 1], leader);
         };
         auto issue_dP = [&](int g) {
             const uint32_t sV = smem_addr(smem + C::kOffV + (g % C::kVStages) * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColdP, sdesc_sw128(sdO + koff, 16, 1024),
-                       sdesc_sw128(sV + koff, 16, 1024), idS, kk > 0);
+                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sdO + koff, 16, 1024),
+                         sdesc_sw128(sV + koff, 16, 1024), idS, kk > 0, leader);
             }
-            mma_commit(&bars->dp_full);
+            mma_commit_w(&bars->dp_full, leader);
         };
         bool ok = true;
         int gt = 0, c = 0;                     // key tiles so far: in the rings, and overall
         for (int j = 0; ok; ++j) {
-            const int b = next_item(j, false);
+            const int b = next_item(j, true);
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const Item it = item(b);
-            if (!mbar_wait(&bars->q_full, j & 1, abort_flag, budget_ns) ||
-                !mbar_wait(&bars->k_full[gt % C::kKStages], (gt / C::kKStages) & 1, abort_flag,
-                           budget_ns)) {
+            if (!mbar_wait_warp(&bars->q_full, j & 1, abort_flag, budget_ns) ||
+                !mbar_wait_warp(&bars->k_full[gt % C::kKStages], (gt / C::kKStages) & 1, abort_flag,
+                                budget_ns)) {
                 ok = false;
                 break;
             }
@@ -339,21 +342,21 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             for (int t = 0; t < it.nkv; ++t, ++c) {
                 const int g = gt + t;
                 // dP(c), once V_j is in and phase B has read dP(c-1).
-                if (!mbar_wait(&bars->v_full[g % C::kVStages], (g / C::kVStages) & 1, abort_flag,
-                               budget_ns) ||
-                    (c > 0 && !mbar_wait(&bars->dp_free, (c - 1) & 1, abort_flag, budget_ns))) {
+                if (!mbar_wait_warp(&bars->v_full[g % C::kVStages], (g / C::kVStages) & 1, abort_flag,
+                                    budget_ns) ||
+                    (c > 0 && !mbar_wait_warp(&bars->dp_free, (c - 1) & 1, abort_flag, budget_ns))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 issue_dP(g);
-                mma_commit(&bars->v_empty[g % C::kVStages]);
-                if (t == it.nkv - 1) mma_commit(&bars->q_empty);   // Q_i, dO_i read for the last time
+                mma_commit_w(&bars->v_empty[g % C::kVStages], leader);
+                if (t == it.nkv - 1) mma_commit_w(&bars->q_empty, leader);   // Q_i, dO_i read for the last time
                 // S(c+1) into the other buffer, whose dS(c-1) the dQ MMA
                 // issued before has read.
                 if (t + 1 < it.nkv) {
-                    if (!mbar_wait(&bars->k_full[(g + 1) % C::kKStages], ((g + 1) / C::kKStages) & 1,
-                                   abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->k_full[(g + 1) % C::kKStages], ((g + 1) / C::kKStages) & 1,
+                                        abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -362,8 +365,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 }
                 // dQ += dS(c) K_j. The item's first one overwrites dQ: the
                 // previous item's epilogue must have read it out.
-                if ((t == 0 && j > 0 && !mbar_wait(&bars->dq_free, (j - 1) & 1, abort_flag, budget_ns)) ||
-                    !mbar_wait(&bars->ds_full, c & 1, abort_flag, budget_ns)) {
+                if ((t == 0 && j > 0 && !mbar_wait_warp(&bars->dq_free, (j - 1) & 1, abort_flag, budget_ns)) ||
+                    !mbar_wait_warp(&bars->ds_full, c & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -372,10 +375,10 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 const uint32_t sbuf = tmem + C::kColS0 + 128 * (c & 1);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)          // keys 16kk .. 16kk+15
-                    mma_ts(tmem + C::kColdQ, sbuf + 64 * (kk >> 2) + 8 * (kk & 3),
-                           sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, t > 0 || kk > 0);
-                mma_commit(&bars->k_empty[g % C::kKStages]);
-                if (t == it.nkv - 1) mma_commit(&bars->dq_done);
+                    mma_ts_w(tmem + C::kColdQ, sbuf + 64 * (kk >> 2) + 8 * (kk & 3),
+                             sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, t > 0 || kk > 0, leader);
+                mma_commit_w(&bars->k_empty[g % C::kKStages], leader);
+                if (t == it.nkv - 1) mma_commit_w(&bars->dq_done, leader);
             }
             gt += it.nkv;
         }
@@ -384,7 +387,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             *abort_flag = 1;
         }
         // Drain: all MMAs issued here complete before TMEM is released.
-        mma_commit(&bars->mma_drain);
+        mma_commit_w(&bars->mma_drain, leader);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
     } else if (!aborted_early && warp < 8) {
         // ------------------------------------------------ elementwise warpgroups

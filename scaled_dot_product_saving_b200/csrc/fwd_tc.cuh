@@ -344,8 +344,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             (void)mbar_wait_timed(&bars->k_full[t % C::kKStages], (t / C::kKStages) & 1, budget_ns);
         for (int t = (v_issued > C::kVStages ? v_issued - C::kVStages : 0); t < v_issued; ++t)
             (void)mbar_wait_timed(&bars->v_full[t % C::kVStages], (t / C::kVStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
+    } else if (!aborted_early && warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
+        // The whole warp walks the loop (waits are warp-wide) and one elected
+        // lane issues the MMAs and commits.
+        const uint32_t leader = elect_leader();
         constexpr uint32_t idS = idesc_bf16_f32(kBM, kBN, 0, 0);
         constexpr uint32_t idO = idesc_bf16_f32(kBM, D, 0, 1);
         auto issue_S = [&](int x, int g) {
@@ -354,10 +357,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColS0 + 128 * x, sdesc_sw128(sQ + koff, 16, 1024),
-                       sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0);
+                mma_ss_w(tmem + C::kColS0 + 128 * x, sdesc_sw128(sQ + koff, 16, 1024),
+                         sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0, leader);
             }
-            mma_commit(&bars->s_full[x]);
+            mma_commit_w(&bars->s_full[x], leader);
         };
         // O_x += P_x V over keys 64h .. 64h+63 of the tile (key tile t of the
         // item, global index g)
@@ -366,21 +369,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int kk = 4 * h + k4;
-                mma_ts(tmem + C::kColO0 + D * x, tmem + C::kColS0 + 128 * x + kk * 8,
-                       sdesc_sw128(sV + kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0));
+                mma_ts_w(tmem + C::kColO0 + D * x, tmem + C::kColS0 + 128 * x + kk * 8,
+                         sdesc_sw128(sV + kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0), leader);
             }
         };
         bool ok = true;
         int gt = 0;
         int cx[2] = {0, 0}, ox[2] = {0, 0}, qx[2] = {0, 0};
         for (int j = 0; ok; ++j) {
-            const int b = next_item(j, false);
+            const int b = next_item(j, true);
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const Item it = item(b);
             // S_x(0) for the active tiles once Q_x and the first K tile are in.
-            if (!mbar_wait(&bars->q_full[0], qx[0] & 1, abort_flag, budget_ns) ||
-                !mbar_wait(&bars->k_full[gt % C::kKStages], (gt / C::kKStages) & 1, abort_flag, budget_ns)) {
+            if (!mbar_wait_warp(&bars->q_full[0], qx[0] & 1, abort_flag, budget_ns) ||
+                !mbar_wait_warp(&bars->k_full[gt % C::kKStages], (gt / C::kKStages) & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
@@ -388,7 +391,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             tc_fence_after();
             issue_S(0, gt);
             if (it.has_b) {
-                if (!mbar_wait(&bars->q_full[1], qx[1] & 1, abort_flag, budget_ns)) {
+                if (!mbar_wait_warp(&bars->q_full[1], qx[1] & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -396,7 +399,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 tc_fence_after();
                 issue_S(1, gt);
             }
-            mma_commit(&bars->k_empty[gt % C::kKStages]);
+            mma_commit_w(&bars->k_empty[gt % C::kKStages], leader);
             for (int t = 0; ok && t < it.num_kv; ++t) {
                 const int g = gt + t;
                 bool v_ready = false, k_ready = false;
@@ -406,13 +409,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (t >= it.nkv[x]) continue;
-                    if (!mbar_wait(&bars->p_half[x], cx[x] & 1, abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->p_half[x], cx[x] & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
                     if (!v_ready) {
-                        if (!mbar_wait(&bars->v_full[g % C::kVStages], (g / C::kVStages) & 1,
-                                       abort_flag, budget_ns)) {
+                        if (!mbar_wait_warp(&bars->v_full[g % C::kVStages], (g / C::kVStages) & 1,
+                                            abort_flag, budget_ns)) {
                             ok = false;
                             break;
                         }
@@ -421,13 +424,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     // The item's first product overwrites O_x: the previous
                     // item's epilogue must have read it out.
                     if (t == 0 && ox[x] > 0 &&
-                        !mbar_wait(&bars->o_free[x], (ox[x] - 1) & 1, abort_flag, budget_ns)) {
+                        !mbar_wait_warp(&bars->o_free[x], (ox[x] - 1) & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     issue_PV(x, t, g, 0);
-                    if (!mbar_wait(&bars->p_full[x], cx[x] & 1, abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->p_full[x], cx[x] & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -436,8 +439,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     ++cx[x];
                     if (t + 1 < it.nkv[x]) {
                         if (!k_ready) {
-                            if (!mbar_wait(&bars->k_full[(g + 1) % C::kKStages], ((g + 1) / C::kKStages) & 1,
-                                           abort_flag, budget_ns)) {
+                            if (!mbar_wait_warp(&bars->k_full[(g + 1) % C::kKStages], ((g + 1) / C::kKStages) & 1,
+                                                abort_flag, budget_ns)) {
                                 ok = false;
                                 break;
                             }
@@ -446,13 +449,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                         }
                         issue_S(x, g + 1);
                     } else {
-                        mma_commit(&bars->o_done[x]);   // last product into O_x
+                        mma_commit_w(&bars->o_done[x], leader);   // last product into O_x
                         ++ox[x];
                     }
                 }
                 if (!ok) break;
-                if (k_ready) mma_commit(&bars->k_empty[(g + 1) % C::kKStages]);
-                mma_commit(&bars->v_empty[g % C::kVStages]);
+                if (k_ready) mma_commit_w(&bars->k_empty[(g + 1) % C::kKStages], leader);
+                mma_commit_w(&bars->v_empty[g % C::kVStages], leader);
             }
             gt += it.num_kv;
         }
@@ -461,7 +464,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             *abort_flag = 1;
         }
         // Drain: all MMAs issued here complete before TMEM is released.
-        mma_commit(&bars->mma_drain);
+        mma_commit_w(&bars->mma_drain, leader);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
     } else if (!aborted_early && warp < 8) {
         // ------------------------------------------------ softmax warpgroups

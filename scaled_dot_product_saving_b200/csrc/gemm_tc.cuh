@@ -118,13 +118,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         }
         for (int kb = (issued > kStages ? issued - kStages : 0); kb < issued; ++kb)
             (void)mbar_wait_timed(&bars->full[kb % kStages], (kb / kStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == 1 && lane == 0) {
+    } else if (!aborted_early && warp == 1) {
         // ------------------------------------------------ MMA issuer
+        // The whole warp walks the loop (waits are warp-wide) and one elected
+        // lane issues the MMAs and commits.
+        const uint32_t leader = elect_leader();
         constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, A_KMAJOR ? 0 : 1, B_KMAJOR ? 0 : 1);
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % kStages;
-            if (!mbar_wait(&bars->full[s], (kb / kStages) & 1, abort_flag, budget_ns)) {
+            if (!mbar_wait_warp(&bars->full[s], (kb / kStages) & 1, abort_flag, budget_ns)) {
                 ok = false;
                 break;
             }
@@ -139,16 +142,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
                                              : sdesc_sw128(sa + kk * 2048, 8192, 1024);
                 const uint64_t db = B_KMAJOR ? sdesc_sw128(sb + kk * 32, 16, 1024)
                                              : sdesc_sw128(sb + kk * 2048, 8192, 1024);
-                mma_ss(tmem, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                mma_ss_w(tmem, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u, leader);
             }
-            mma_commit(&bars->empty[s]);
+            mma_commit_w(&bars->empty[s], leader);
         }
-        if (ok) mma_commit(&bars->acc_full);
+        if (ok) mma_commit_w(&bars->acc_full, leader);
         else {
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
-        mma_commit(&bars->mma_drain);
+        mma_commit_w(&bars->mma_drain, leader);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
     } else if (!aborted_early && warp >= 2) {
         // ------------------------------------------------ epilogue

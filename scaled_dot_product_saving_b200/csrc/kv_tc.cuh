@@ -364,8 +364,11 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         if (kv_issued > 0) (void)mbar_wait_timed(&bars->kv_full, (kv_issued - 1) & 1, budget_ns);
         for (int t = (g > C::kStages ? g - C::kStages : 0); t < g; ++t)
             (void)mbar_wait_timed(&bars->q_full[t % C::kStages], (t / C::kStages) & 1, budget_ns);
-    } else if (!aborted_early && warp == kWarpMma && lane == 0) {
+    } else if (!aborted_early && warp == kWarpMma) {
         // ------------------------------------------------ MMA issuer
+        // The whole warp walks the loop (waits are warp-wide) and one elected
+        // lane issues the MMAs and commits.
+        const uint32_t leader = elect_leader();
         constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
         constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
         const uint32_t sK = smem_addr(smem + C::kOffK);
@@ -374,16 +377,16 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
         // s_full / dp_full report them.
         auto issue_S = [&](int g) -> bool {
             const int s = g % C::kStages;
-            if (!mbar_wait(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
+            if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
             tc_fence_after();
             const uint32_t sQ = smem_addr(smem + C::kOffQ + s * C::kTileBytes);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
-                       sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0);
+                mma_ss_w(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
+                         sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0, leader);
             }
-            mma_commit(&bars->s_full);
+            mma_commit_w(&bars->s_full, leader);
             return true;
         };
         auto issue_dP = [&](int g) {
@@ -391,19 +394,19 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                       sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0);
+                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                         sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0, leader);
             }
-            mma_commit(&bars->dp_full);
+            mma_commit_w(&bars->dp_full, leader);
         };
         bool ok = true;
         int g = 0;
         for (int j = 0; ok; ++j) {
-            const int b = next_item(j, false);
+            const int b = next_item(j, true);
             if (b == -1) break;
             if (b < 0) { ok = false; break; }
             const int T = item(b).T;
-            if (!mbar_wait(&bars->kv_full, j & 1, abort_flag, budget_ns) || !issue_S(g)) {
+            if (!mbar_wait_warp(&bars->kv_full, j & 1, abort_flag, budget_ns) || !issue_S(g)) {
                 ok = false;
                 break;
             }
@@ -415,7 +418,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 // The item's first dV MMA overwrites the accumulators: the
                 // previous item's epilogue must have read them out.
                 if (t == 0 && j > 0 &&
-                    !mbar_wait(&bars->acc_free, (j - 1) & 1, abort_flag, budget_ns)) {
+                    !mbar_wait_warp(&bars->acc_free, (j - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -425,7 +428,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 bool first = (t == 0);
                 for (int ci = 0; ci < kChunks; ++ci) {
                     const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
-                    if (!mbar_wait(&bars->p_chunk[c], g & 1, abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->p_chunk[c], g & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -433,8 +436,8 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
-                        mma_ts(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
-                               sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                        mma_ts_w(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
+                                 sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
                 }
@@ -445,7 +448,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                 first = (t == 0);
                 for (int ci = 0; ci < kChunks; ++ci) {
                     const int c = (ci >> 1) | ((ci & 1) << 1);
-                    if (!mbar_wait(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
+                    if (!mbar_wait_warp(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
                         ok = false;
                         break;
                     }
@@ -453,18 +456,18 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;
-                        mma_ts(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
-                               sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first);
+                        mma_ts_w(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
+                                 sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
                 }
                 if (!ok) break;
-                mma_commit(&bars->q_empty[s]);
+                mma_commit_w(&bars->q_empty[s], leader);
                 // dP^T(g+1): every MMA that reads dS^T(g) has been issued.
                 if (t + 1 < T) issue_dP(g + 1);
                 if (t == T - 1) {
-                    mma_commit(&bars->acc_done);
-                    mma_commit(&bars->kv_empty);      // K_j, V_j free once these complete
+                    mma_commit_w(&bars->acc_done, leader);
+                    mma_commit_w(&bars->kv_empty, leader);      // K_j, V_j free once these complete
                 }
             }
         }
@@ -472,7 +475,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
             record_device_error(kErrTimeout);
             *abort_flag = 1;
         }
-        mma_commit(&bars->mma_drain);
+        mma_commit_w(&bars->mma_drain, leader);
         (void)mbar_wait_timed(&bars->mma_drain, 0, budget_ns);
     } else if (!aborted_early && warp < 8) {
         // ------------------------------------------------ P / dS warpgroups

@@ -63,15 +63,19 @@ def scheduler_heads(w: synth.Workload):
     element: the first, middle and last head of every head group of the
     tensor-core backward's and forward's schedules (groups of about 256 work
     items: 128 keys per backward item, two 128-row query tiles per forward
-    item), so that every group is checked. Heads are numbered b*H + h."""
+    item; when causal the backward merges its last two groups into one), so
+    that every group is checked. Heads are numbered b*H + h."""
     BH = w.B * w.H
     picked = set()
     num_kt = -(-w.m // 128)
     num_pairs = -(-(-(-w.n // 128)) // 2)
-    for items_per_head in (num_kt, num_pairs):
+    for items_per_head, merge_last in ((num_kt, w.causal), (num_pairs, False)):
         hg = max(1, min(BH, 256 // items_per_head))
-        for g0 in range(0, BH, hg):
-            last = min(BH, g0 + hg) - 1
+        starts = list(range(0, BH, hg))
+        if merge_last and len(starts) >= 2:
+            starts.pop()
+        for i, g0 in enumerate(starts):
+            last = (starts[i + 1] if i + 1 < len(starts) else BH) - 1
             picked.update({g0, (g0 + last) // 2, last})
     return [(x // w.H, x % w.H) for x in sorted(picked)]
 
