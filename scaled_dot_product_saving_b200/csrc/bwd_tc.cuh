@@ -64,7 +64,11 @@
 // pipe runs MMAs in issue order, so the dQ MMA, issued after the last dV MMA,
 // overwrites P^T only once it has been read; the next tile's dP^T MMA is
 // issued before the dQ drain is awaited and only its S^T MMA waits for it.
-// d = 64: dV [0,64) dK [64,128) S^T [128,256) dP^T [256,384) dQ [384,448).
+// d = 64: dV [0,64) dK [64,128), then per 64-query half h (chunks 2h, 2h+1)
+// S^T at 128 + 128h and dP^T 64 columns after it, dQ [384,448). Each P/dS
+// warpgroup owns one half: the MMA thread issues the half's next S^T/dP^T
+// as soon as it has issued the half's last dV/dK k-steps, so one warpgroup
+// works on tile t+1 while the MMAs of the other's half of tile t run.
 #pragma once
 
 #include "sm100.cuh"
@@ -134,13 +138,25 @@ struct Cfg {
     static constexpr int kPanels = D / 64;
     static constexpr int kTileBytes = 128 * D * 2;     // a 128-row bf16 tile
     static constexpr int kPanelBytes = 128 * 128;      // 128 rows x 128 B
+    // d = 64: each P/dS warpgroup runs its own 64-query half of every tile
+    // (S^T/dP^T of the half in TMEM columns of its own, signalled on its own
+    // barrier), and dQ is staged in a buffer of its own rather than in the dS
+    // tile; d = 128 has neither the TMEM nor the shared memory for that.
+    static constexpr bool kSplit = (D == 64);
     static constexpr int kOffK = 0;                    // K/V buffer b: K at kOffK + b * kKVBytes,
     static constexpr int kOffV = kOffK + kTileBytes;   // V kTileBytes after it
     static constexpr int kKVBytes = 2 * kTileBytes;
     static constexpr int kOffQ = kKV * kKVBytes;
     static constexpr int kOffdO = kOffQ + kStages * kTileBytes;
     static constexpr int kOffdS = kOffdO + kStages * kTileBytes;   // 128 keys x 128 queries
-    static constexpr int kOffLse = kOffdS + 128 * 128 * 2;
+    // dQ staging, per warp of the dQ warpgroup: 32-row x 32-column fp32
+    // buffers (4 KB each, 128B-swizzled) used in turn by the row's D/32
+    // segments. d = 128: two per warp, in the dS tile (free between the dQ
+    // MMA and the next tile's dS); d = 64: one per warp, after the dS tile.
+    static constexpr int kStageBufs = kSplit ? 1 : 2;
+    static constexpr int kStageWarpBytes = kStageBufs * 4096;
+    static constexpr int kOffStage = kSplit ? kOffdS + 128 * 128 * 2 : kOffdS;
+    static constexpr int kOffLse = kSplit ? kOffStage + 4 * kStageWarpBytes : kOffdS + 128 * 128 * 2;
     static constexpr int kOffDd = kOffLse + kStages * kBM * 4;
     static constexpr int kOffBar = kOffDd + kStages * kBM * 4;
     static constexpr int kSmemBytes = kOffBar + 512;
@@ -148,23 +164,24 @@ struct Cfg {
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColdV = 0;
     static constexpr uint32_t kColdK = D;
-    static constexpr uint32_t kColS = 2 * D;
-    static constexpr uint32_t kColdP = 2 * D + 128;
-    static constexpr uint32_t kColP = kColS;          // bf16 P^T over S^T
-    static constexpr uint32_t kColdS = kColdP;        // bf16 dS^T over dP^T
-    static constexpr uint32_t kColdQ = kAlias ? kColS : 2 * D + 256;
-    // dQ staging through the dS tile: per warp, two 32-row x 32-column fp32
-    // buffers (4 KB each, 128B-swizzled) that alternate over the row's D/32
-    // segments.
-    static constexpr int kStageWarpBytes = 8192;
+    // S^T and dP^T of the 32-query chunk c (chunks 2h, 2h+1 form half h).
+    // bf16 P^T / dS^T are written over the first 16 of the chunk's columns.
+    // d = 128: S^T [256,384), dP^T [384,512). d = 64, per half h: S^T at
+    // 128 + 128h, dP^T 64 columns after it.
+    static constexpr uint32_t col_s(int c) {
+        return kSplit ? 2 * D + (c >> 1) * 128 + (c & 1) * 32 : 2 * D + 32 * c;
+    }
+    static constexpr uint32_t col_dp(int c) { return col_s(c) + (kSplit ? 64 : 128); }
+    static constexpr uint32_t kColdQ = kAlias ? 2 * D : 2 * D + 256;
 };
+static_assert(Cfg<64>::kSmemBytes <= 232448 && Cfg<128>::kSmemBytes <= 232448, "shared memory");
 
 struct Bars {
     uint64_t kv_full[2];
     uint64_t kv_empty[2];   // the item's last MMA has read K_j, V_j of buffer b
     uint64_t q_full[4];
     uint64_t q_empty[4];
-    uint64_t s_full;
+    uint64_t s_full[2];     // S^T, dP^T of the tile (d = 64: of half h) are in TMEM
     uint64_t ds_chunk[kChunks];
     uint64_t dq_full;
     uint64_t dq_free;
@@ -370,7 +387,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             mbar_init(&bars->q_full[s], 1);
             mbar_init(&bars->q_empty[s], 1);
         }
-        mbar_init(&bars->s_full, 1);
+        for (int h = 0; h < 2; ++h) mbar_init(&bars->s_full[h], 1);
         for (int c = 0; c < kChunks; ++c) mbar_init(&bars->ds_chunk[c], 128);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_free, 128);
@@ -538,9 +555,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // The whole warp walks the loop (waits are warp-wide) and one elected
         // lane issues the MMAs and commits.
         const uint32_t leader = elect_leader();
-        constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);   // S^T, dP^T
-        constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);     // dV, dK
-        constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 1, 1);      // dQ
+        constexpr uint32_t idSP = idesc_bf16_f32(kBN, kBM, 0, 0);       // S^T, dP^T
+        constexpr uint32_t idHalf = idesc_bf16_f32(kBN, kBM / 2, 0, 0); // ... of a 64-query half
+        constexpr uint32_t idKV = idesc_bf16_f32(kBN, D, 0, 1);         // dV, dK
+        constexpr uint32_t idQ = idesc_bf16_f32(kBM, D, 1, 1);          // dQ
         uint32_t sK = smem_addr(smem + C::kOffK), sV = smem_addr(smem + C::kOffV);   // per item
         const uint32_t sdS = smem_addr(smem + C::kOffdS);
         // dP^T(g) = V dO(g)^T once Q/dO(g) are in; its columns are free once
@@ -553,7 +571,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
+                mma_ss_w(tmem + C::col_dp(0), sdesc_sw128(sV + koff, 16, 1024),
                          sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0, leader);
             }
             return true;
@@ -570,10 +588,35 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
+                mma_ss_w(tmem + C::col_s(0), sdesc_sw128(sK + koff, 16, 1024),
                          sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0, leader);
             }
-            mma_commit_w(&bars->s_full, leader);
+            mma_commit_w(&bars->s_full[0], leader);
+            return true;
+        };
+        // d = 64: dP^T and S^T of the 64-query half h of tile g (queries
+        // 64h.., rows 64h.. of the Q/dO tiles, 8 KB in); s_full[h] reports
+        // both. Their columns were last read by the half's dV/dK MMAs of the
+        // previous tile, issued earlier.
+        auto issue_half = [&](int g, int h) -> bool {
+            const int s = g % C::kStages;
+            if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
+            tc_fence_after();
+            const uint32_t sQh = smem_addr(smem + C::kOffQ + s * C::kTileBytes) + h * 8192;
+            const uint32_t sdOh = smem_addr(smem + C::kOffdO + s * C::kTileBytes) + h * 8192;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                mma_ss_w(tmem + C::col_dp(2 * h), sdesc_sw128(sV + koff, 16, 1024),
+                         sdesc_sw128(sdOh + koff, 16, 1024), idHalf, kk > 0, leader);
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+                mma_ss_w(tmem + C::col_s(2 * h), sdesc_sw128(sK + koff, 16, 1024),
+                         sdesc_sw128(sQh + koff, 16, 1024), idHalf, kk > 0, leader);
+            }
+            mma_commit_w(&bars->s_full[h], leader);
             return true;
         };
         bool ok = true;
@@ -590,20 +633,18 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             }
             sK = smem_addr(smem + C::kOffK + kb * C::kKVBytes);
             sV = smem_addr(smem + C::kOffV + kb * C::kKVBytes);
-            // At d = 64 (dQ in columns of its own) the next tile's dP^T and S^T
-            // are issued right after this tile's dV/dK MMAs, before the dQ MMA
-            // waits for the dS tile, so the P/dS warps start on tile t+1 while
-            // dS(t) reaches shared memory. At d = 128 the dQ MMA goes first:
-            // its result paces the dQ reduce-adds, whose staging holds the dS
-            // tile (issuing dP^T first measured 8 % slower).
-            bool ahead = false;
+            // d = 128: per tile dP^T, S^T, the dV/dK k-steps chunk by chunk,
+            // then dQ; the next tile's S^T overwrites dQ's columns, so it waits
+            // for the dQ warpgroup to read them out. d = 64: each half's next
+            // dP^T/S^T is issued as soon as the half's last dV/dK k-steps are,
+            // so a P/dS warpgroup starts on its half of tile t+1 while the
+            // other warpgroup still works on tile t.
+            if (C::kSplit && (!issue_half(g, 0) || !issue_half(g, 1))) { ok = false; break; }
             for (int t = 0; t < T; ++t, ++g) {
                 const int s = g % C::kStages;
                 const uint32_t sQ = smem_addr(smem + C::kOffQ + s * C::kTileBytes);
                 const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
-                if (!ahead && !issue_dP(g)) { ok = false; break; }
-                if (!ahead && !issue_S(g)) { ok = false; break; }
-                ahead = false;
+                if (!C::kSplit && (!issue_dP(g) || !issue_S(g))) { ok = false; break; }
                 // The item's first dV/dK MMAs overwrite the accumulators: the
                 // previous item's epilogue must have read them out.
                 if (t == 0 && j > 0 &&
@@ -625,23 +666,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
-                        mma_ts_w(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
+                        mma_ts_w(tmem + C::kColdV, tmem + C::col_s(c) + 8 * h,
                                  sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
-                        mma_ts_w(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
+                        mma_ts_w(tmem + C::kColdK, tmem + C::col_dp(c) + 8 * h,
                                  sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
+                    }
+                    if (C::kSplit && (c & 1) && t + 1 < T && !issue_half(g + 1, c >> 1)) {
+                        ok = false;
+                        break;
                     }
                 }
                 if (!ok) break;
                 mma_commit_w(&bars->q_empty[s], leader);
                 if (t == T - 1) mma_commit_w(&bars->acc_done, leader);
-                if (!C::kAlias && t + 1 < T) {
-                    if (!issue_dP(g + 1) || !issue_S(g + 1)) {
-                        ok = false;
-                        break;
-                    }
-                    ahead = true;
-                }
                 if (!C::kAlias && g > 0 &&
                     !mbar_wait_warp(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
                     ok = false;
@@ -686,7 +724,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 const int s = g % C::kStages;
                 const int q0 = (it.first_qt + t) * kBM;
                 if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns) ||
-                    !mbar_wait_warp(&bars->s_full, g & 1, abort_flag, budget_ns)) {
+                    !mbar_wait_warp(&bars->s_full[C::kSplit ? grp : 0], g & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
                 }
@@ -709,8 +747,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 uint32_t ds0[16], ds1[16];
                 uint32_t sA[16], pA[16], sB[16], pB[16];
                 const int cbase = 2 * grp;
-                tmem_ld16(tl + C::kColS + cbase * 32, sA);
-                tmem_ld16(tl + C::kColdP + cbase * 32, pA);
+                tmem_ld16(tl + C::col_s(cbase), sA);
+                tmem_ld16(tl + C::col_dp(cbase), pA);
                 tmem_ld_wait();
 #pragma unroll
                 for (int hc = 0; hc < 4; ++hc) {
@@ -721,13 +759,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     uint32_t (&snxt)[16] = (hc & 1) ? sA : sB;
                     uint32_t (&pnxt)[16] = (hc & 1) ? pA : pB;
                     if (hc < 3) {
-                        const int qn = 32 * (cbase + ((hc + 1) >> 1)) + 16 * ((hc + 1) & 1);
-                        tmem_ld16(tl + C::kColS + qn, snxt);
-                        tmem_ld16(tl + C::kColdP + qn, pnxt);
+                        const int cn = cbase + ((hc + 1) >> 1), hn = (hc + 1) & 1;
+                        tmem_ld16(tl + C::col_s(cn) + 16 * hn, snxt);
+                        tmem_ld16(tl + C::col_dp(cn) + 16 * hn, pnxt);
                     }
                     uint32_t* dk = ((hc >> 1) ? ds1 : ds0) + 8 * half;
-                    const uint32_t pcol = tl + C::kColP + 32 * c + 8 * half;
-                    const uint32_t dscol = tl + C::kColdS + 32 * c + 8 * half;
+                    const uint32_t pcol = tl + C::col_s(c) + 8 * half;
+                    const uint32_t dscol = tl + C::col_dp(c) + 8 * half;
                     if (masked)
                         pds_half<true>(qcol, scur, pcur, lse_s, dd_s, below, scale, scale_log2, pcol,
                                        dscol, dk);
@@ -741,10 +779,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     }
                     if (hc < 3) tmem_ld_wait();
                 }
-                // The dS tile doubles as the dQ warpgroup's staging buffer for
-                // the previous tile: write it once the TMA has read that.
-                if (g > 0 &&
-                    !mbar_wait_warp(&bars->ds_smem_free, (g - 1) & 1, abort_flag, budget_ns)) {
+                // d = 128: the dS tile doubles as the dQ warpgroup's staging
+                // buffer for the previous tile: write it once the TMA has read
+                // that. d = 64: once the previous tile's dQ MMA has read it.
+                if (g > 0 && !(C::kSplit ? mbar_wait_warp(&bars->dq_full, (g - 1) & 1, abort_flag, budget_ns)
+                                         : mbar_wait_warp(&bars->ds_smem_free, (g - 1) & 1, abort_flag,
+                                                          budget_ns))) {
                     ok = false;
                     break;
                 }
@@ -811,15 +851,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         }
     } else if (!aborted_early && warp >= kWarpDq && warp < kWarpDq + 4) {
         // ------------------------------------------------ dQ warpgroup
-        // Thread r owns query row r of the tile (its TMEM lane). Once the dQ
-        // MMA has completed, the dS tile is free until the P/dS warpgroup
-        // writes the next tile's dS. Each warp stages its 32 rows there one
-        // 32-column segment at a time, in the 128-byte swizzled layout of the
-        // accumulator's tensor map, and one lane hands each segment to the
-        // TMA engine as a tiled reduce-add; rows past n are clipped by the TMA.
+        // Thread r owns query row r of the tile (its TMEM lane). Each warp
+        // stages its 32 rows one 32-column segment at a time, in the 128-byte
+        // swizzled layout of the accumulator's tensor map, and one lane hands
+        // each segment to the TMA engine as a tiled reduce-add; rows past n
+        // are clipped by the TMA. d = 128 stages in the dS tile, free from
+        // the dQ MMA's completion until the P/dS warpgroups write the next
+        // tile's dS; d = 64 in a buffer of its own.
         const int wq = warp & 3;
         const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
-        uint8_t* stage = smem + C::kOffdS + wq * C::kStageWarpBytes;
+        uint8_t* stage = smem + C::kOffStage + wq * C::kStageWarpBytes;
         bool ok = true;
         int g = 0;
         for (int j = 0; ok; ++j) {
@@ -851,9 +892,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
                 for (int sg = 0; sg < kSegs; ++sg) {                  // columns 32sg..32sg+31
                     uint32_t (&v)[32] = (sg & 1) ? vb : va;
-                    uint8_t* buf = stage + (sg & 1) * 4096;
-                    if (sg >= 2) {
-                        if (lane == 0) bulk_wait_group_read1();       // buffer's previous segment read
+                    uint8_t* buf = stage + (sg % C::kStageBufs) * 4096;
+                    if (sg >= C::kStageBufs) {
+                        if (lane == 0) {                              // buffer's previous segment read
+                            if (C::kStageBufs == 2) bulk_wait_group_read1();
+                            else bulk_wait_group_read0();
+                        }
                         __syncwarp();
                     }
 #pragma unroll
@@ -877,7 +921,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 }
                 if (lane == 0) bulk_wait_group_read0();
                 __syncwarp();
-                mbar_arrive(&bars->ds_smem_free);
+                if (!C::kSplit) mbar_arrive(&bars->ds_smem_free);
             }
             if (!ok) break;
             // Every partial of this item has been handed to the TMA: once they
