@@ -391,7 +391,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         for (int c = 0; c < kChunks; ++c) mbar_init(&bars->ds_chunk[c], 128);
         mbar_init(&bars->dq_full, 1);
         mbar_init(&bars->dq_free, 128);
-        mbar_init(&bars->ds_smem_full, 256);
+        // d = 64: the dQ warpgroup's "dQ read out of TMEM" arrives here too,
+        // so one wait covers both conditions of the next dQ MMA.
+        mbar_init(&bars->ds_smem_full, C::kSplit ? 256 + 128 : 256);
         mbar_init(&bars->ds_smem_free, 128);
         mbar_init(&bars->acc_done, 1);
         mbar_init(&bars->acc_free, 256);
@@ -600,7 +602,9 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         // previous tile, issued earlier.
         auto issue_half = [&](int g, int h) -> bool {
             const int s = g % C::kStages;
-            if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
+            // Half 1 always follows half 0 of the same tile, whose wait saw Q/dO in.
+            if (h == 0 && !mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns))
+                return false;
             tc_fence_after();
             const uint32_t sQh = smem_addr(smem + C::kOffQ + s * C::kTileBytes) + h * 8192;
             const uint32_t sdOh = smem_addr(smem + C::kOffdO + s * C::kTileBytes) + h * 8192;
@@ -652,17 +656,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     ok = false;
                     break;
                 }
-                // dV += P^T dO and dK += dS^T Q, 32 queries (two k-steps) per
-                // chunk as soon as a P/dS warpgroup has written that chunk; the
-                // two warpgroups finish chunks 0 and 2 first, then 1 and 3.
+                // dV += P^T dO and dK += dS^T Q, two k-steps per 32-query chunk.
+                // d = 128: chunk by chunk as soon as a P/dS warpgroup has written
+                // it; the two warpgroups finish chunks 0 and 2 first, then 1
+                // and 3. d = 64: a half at a time (its warpgroup signals chunk
+                // 2h+1 after chunk 2h), then the half's next S^T/dP^T.
                 bool first = (t == 0);
-                for (int ci = 0; ci < kChunks; ++ci) {
-                    const int c = (ci >> 1) | ((ci & 1) << 1);        // 0, 2, 1, 3
-                    if (!mbar_wait_warp(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                auto issue_chunk = [&](int c) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
@@ -672,19 +672,36 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                                  sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
-                    if (C::kSplit && (c & 1) && t + 1 < T && !issue_half(g + 1, c >> 1)) {
-                        ok = false;
-                        break;
+                };
+                if (C::kSplit) {
+                    for (int h = 0; h < 2; ++h) {
+                        if (!mbar_wait_warp(&bars->ds_chunk[2 * h + 1], g & 1, abort_flag, budget_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_chunk(2 * h);
+                        issue_chunk(2 * h + 1);
+                        if (t + 1 < T && !issue_half(g + 1, h)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                } else {
+                    for (int ci = 0; ci < kChunks; ++ci) {
+                        const int c = (ci >> 1) | ((ci & 1) << 1);    // 0, 2, 1, 3
+                        if (!mbar_wait_warp(&bars->ds_chunk[c], g & 1, abort_flag, budget_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_chunk(c);
                     }
                 }
                 if (!ok) break;
                 mma_commit_w(&bars->q_empty[s], leader);
                 if (t == T - 1) mma_commit_w(&bars->acc_done, leader);
-                if (!C::kAlias && g > 0 &&
-                    !mbar_wait_warp(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns)) {
-                    ok = false;
-                    break;
-                }
+                // dS(g) in shared memory (and, d = 64, dQ(g-1) read out of TMEM).
                 if (!mbar_wait_warp(&bars->ds_smem_full, g & 1, abort_flag, budget_ns)) {
                     ok = false;
                     break;
@@ -861,6 +878,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         const int wq = warp & 3;
         const uint32_t tl = tmem + (uint32_t(wq * 32) << 16);
         uint8_t* stage = smem + C::kOffStage + wq * C::kStageWarpBytes;
+        // d = 64: "dQ read out" goes to the barrier of the next dQ MMA, which
+        // also counts the dS stores; the first dQ MMA has nothing to wait for.
+        uint64_t* dq_read = C::kSplit ? &bars->ds_smem_full : &bars->dq_free;
+        if (C::kSplit) mbar_arrive(dq_read);
         bool ok = true;
         int g = 0;
         for (int j = 0; ok; ++j) {
@@ -887,7 +908,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 tmem_ld_wait();
                 if (kSegs == 2) {
                     tc_fence_before();
-                    mbar_arrive(&bars->dq_free);
+                    mbar_arrive(dq_read);
                 }
 #pragma unroll
                 for (int sg = 0; sg < kSegs; ++sg) {                  // columns 32sg..32sg+31
@@ -909,7 +930,7 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                         if (sg + 3 == kSegs) {
                             tmem_ld_wait();
                             tc_fence_before();
-                            mbar_arrive(&bars->dq_free);
+                            mbar_arrive(dq_read);
                         }
                     }
                     fence_proxy_async_smem();
