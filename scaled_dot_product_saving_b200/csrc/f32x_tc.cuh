@@ -40,7 +40,10 @@
 // The backward is two passes that each recompute S and dP, so that neither
 // needs a transposed copy of dS in shared memory (three pieces of a 128 x 128
 // tile would not fit beside the operands). Streamed tiles are double
-// buffered: the loads of tile t + 2 run while the MMAs of tile t + 1 do.
+// buffered. In both passes the next tile's S/dP MMAs are issued before this
+// tile's dV/dK (dQ) MMAs, so the elementwise step of the next tile runs
+// under them; its pieces go to TMEM once they are done, when the buffer of
+// the tile before is also reloaded.
 //
 // The backward takes D multiplied by the scale and the LSE in base 2, from
 // the preprocess kernel (padded to whole 128-row tiles: LSE = +inf and D = 0
@@ -466,7 +469,10 @@ __device__ __forceinline__ void split32_to_tmem(const uint32_t (&v)[32], uint32_
     }
 }
 
-// acc[0..31] += the 32 fp32 columns of this lane at taddr.
+
+// acc[0..31] += the 32 fp32 columns of this lane at taddr. The tiles' dV,
+// dK and dQ are summed here in fp32 rather than by accumulating MMAs across
+// tiles in TMEM, which measured above the fp32 parity bar.
 __device__ __forceinline__ void add_tmem32(uint32_t taddr, float (&acc)[32]) {
     uint32_t r[32];
     tmem_ld32(taddr, r);
@@ -474,7 +480,6 @@ __device__ __forceinline__ void add_tmem32(uint32_t taddr, float (&acc)[32]) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) acc[c] += __uint_as_float(r[c]);
 }
-
 
 // ---------------------------------------------------- dK and dV pass
 // TMEM columns: S^T (64), dP^T (64), this tile's dV (64) and dK (64), P^T
@@ -575,19 +580,24 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
         mma6_ss(tmem + kKvColdP, sV, kBigPiece, sdO, kSmallPiece, kIdSS);
         mma_commit(&bars->bar_a);
     }
+
+    // Per query tile: S^T/dP^T(idx) -> P^T, dS^T in registers -> (once the
+    // previous tile's dV/dK MMAs are done with the pieces) split into TMEM ->
+    // S^T/dP^T(idx+1), then dV/dK(idx). S^T/dP^T of the next tile are issued
+    // first, so the P/dS arithmetic of tile idx+1 runs under the dV/dK MMAs
+    // of tile idx; each tile's dV and dK are added into registers.
     float acc_v[32], acc_k[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) acc_v[c] = acc_k[c] = 0.f;
-
     for (int idx = 0; ok && idx < T; ++idx) {
         const int buf = idx & 1;
         const int qb = (i0 + idx) * kSmall + 32 * half;     // first query of this half
-        const bool got = mbar_wait_warp(&bars->bar_a, idx & 1, &never, budget_ns);
+        bool got = mbar_wait_warp(&bars->bar_a, idx & 1, &never, budget_ns);
+        uint32_t sr[32], pr[32];
         if (got) {
             tc_fence_after();
             const float* Lrow = sRow + buf * 128 + 32 * half;
             const float* Drow = Lrow + kSmall;
-            uint32_t sr[32], pr[32];
             tmem_ld32(tl + kKvColS, sr);
             tmem_ld32(tl + kKvColdP, pr);
             tmem_ld_wait(sr);
@@ -599,6 +609,24 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
                 sr[c] = __float_as_uint(pv);
                 pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -Drow[c]));
             }
+        }
+        // The previous tile's dV/dK MMAs have read the P^T/dS^T pieces and
+        // Q, dO of buffer buf^1: tile idx + 1 goes there, idx + 2 starts
+        // arriving.
+        if (got && idx > 0) {
+            got = mbar_wait_warp(&bars->bar_b, (idx - 1) & 1, &never, budget_ns);
+            if (got) {
+                tc_fence_after();
+                add_tmem32(tl + kKvColdV, acc_v);
+                add_tmem32(tl + kKvColdK, acc_k);
+            }
+            if (got && idx + 1 < T) {
+                split_q(buf ^ 1);
+                fence_proxy_async_smem();
+                if (idx + 2 < T) fetch_q(idx + 2);
+            }
+        }
+        if (got) {
             // this half's 32 queries are K elements 32 half .. +31: columns 16 half ..
             split32_to_tmem(sr, tl - 32 * half + kKvColP + 16 * half);
             split32_to_tmem(pr, tl - 32 * half + kKvColdS + 16 * half);
@@ -611,9 +639,6 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
         }
         if (tid == 0) {
             tc_fence_after();
-            mma6_ts(tmem + kKvColdV, tmem + kKvColP, sdO + buf * kSmallTile, kIdTS, false);
-            mma6_ts(tmem + kKvColdK, tmem + kKvColdS, sQ + buf * kSmallTile, kIdTS, false);
-            mma_commit(&bars->bar_b);
             if (idx + 1 < T) {
                 mma6_ss(tmem + kKvColS, sK, kBigPiece, sQ + (buf ^ 1) * kSmallTile, kSmallPiece,
                         kIdSS);
@@ -621,35 +646,25 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
                         kIdSS);
                 mma_commit(&bars->bar_a);
             }
-        }
-        const bool got2 = mbar_wait_warp(&bars->bar_b, idx & 1, &never, budget_ns);
-        if (got2) {
-            tc_fence_after();
-            add_tmem32(tl + kKvColdV, acc_v);
-            add_tmem32(tl + kKvColdK, acc_k);
-            // Q_i, dO_i, their LSE and D are free once dV, dK of this tile
-            // are done: tile idx + 2 goes there, tile idx + 3 starts arriving.
-            if (idx + 2 < T) {
-                split_q(buf);
-                fence_proxy_async_smem();
-                if (idx + 3 < T) fetch_q(idx + 3);
-            }
-        }
-        tc_fence_before();
-        if (__syncthreads_or(!got2)) {
-            ok = false;
-            break;
+            mma6_ts(tmem + kKvColdV, tmem + kKvColP, sdO + buf * kSmallTile, kIdTS, false);
+            mma6_ts(tmem + kKvColdK, tmem + kKvColdS, sQ + buf * kSmallTile, kIdTS, false);
+            mma_commit(&bars->bar_b);
         }
     }
 
     if (ok) {
-        if (krow < m) {
-            store_half(dV + (size_t(bh) * m + krow) * dv, 32 * half, acc_v, dv);
-            store_half(dK + (size_t(bh) * m + krow) * d, 32 * half, acc_k, d);
+        ok = mbar_wait_warp(&bars->bar_b, (T - 1) & 1, &never, budget_ns);
+        if (ok) {
+            tc_fence_after();
+            add_tmem32(tl + kKvColdV, acc_v);
+            add_tmem32(tl + kKvColdK, acc_k);
+            if (krow < m) {
+                store_half(dV + (size_t(bh) * m + krow) * dv, 32 * half, acc_v, dv);
+                store_half(dK + (size_t(bh) * m + krow) * d, 32 * half, acc_k, d);
+            }
         }
-    } else if (tid == 0) {
-        record_device_error(kErrTimeout);
     }
+    if (!ok && tid == 0) record_device_error(kErrTimeout);
     teardown(bars, tmem, kKvTmemCols, budget_ns);
 }
 
@@ -730,17 +745,21 @@ dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
         mma6_ss(tmem + kDqColdP, sdO, kBigPiece, sV, kSmallPiece, kIdSS);
         mma_commit(&bars->bar_a);
     }
+
+    // Per key tile, as in the dK/dV pass: S/dP(j) -> dS in registers ->
+    // (once dQ(j-1) has read the dS pieces and K of buffer buf^1) split into
+    // TMEM -> S/dP(j+1), then dQ(j); each tile's dQ is added into registers.
     float acc[32];
 #pragma unroll
     for (int c = 0; c < 32; ++c) acc[c] = 0.f;
-
     for (int j = 0; ok && j < T; ++j) {
         const int buf = j & 1;
         const int kb = j * kSmall + 32 * half;               // first key of this half
-        const bool got = mbar_wait_warp(&bars->bar_a, j & 1, &never, budget_ns);
+        bool got = mbar_wait_warp(&bars->bar_a, j & 1, &never, budget_ns);
+        uint32_t pr[32];
         if (got) {
             tc_fence_after();
-            uint32_t sr[32], pr[32];
+            uint32_t sr[32];
             tmem_ld32(tl + kDqColS, sr);
             tmem_ld32(tl + kDqColdP, pr);
             tmem_ld_wait(sr);
@@ -752,6 +771,23 @@ dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
                 if (key >= mk || (causal && key > row)) pv = 0.f;
                 pr[c] = __float_as_uint(pv * fmaf(__uint_as_float(pr[c]), scale, -dd));
             }
+        }
+        // K, V of buffer buf^1 (tile j-1) and the dS pieces are free once
+        // dQ(j-1) is done: tile j + 1 goes there, j + 2 starts arriving.
+        if (got && j > 0) {
+            got = mbar_wait_warp(&bars->bar_b, (j - 1) & 1, &never, budget_ns);
+            if (got) {
+                tc_fence_after();
+                add_tmem32(tl + kDqColdQ, acc);
+            }
+            if (got && j + 1 < T) {
+                split_staged<kSmall, kBwdThreads>(stK, smem + kDqOffK + (buf ^ 1) * kSmallTile, tid);
+                split_staged<kSmall, kBwdThreads>(stV, smem + kDqOffV + (buf ^ 1) * kSmallTile, tid);
+                fence_proxy_async_smem();
+                if (j + 2 < T) fetch_kv(j + 2);
+            }
+        }
+        if (got) {
             split32_to_tmem(pr, tl - 32 * half + kDqColdS + 16 * half);
             tmem_st_wait();
         }
@@ -762,8 +798,6 @@ dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
         }
         if (tid == 0) {
             tc_fence_after();
-            mma6_ts(tmem + kDqColdQ, tmem + kDqColdS, sK + buf * kSmallTile, kIdTS, false);
-            mma_commit(&bars->bar_b);
             if (j + 1 < T) {
                 mma6_ss(tmem + kDqColS, sQ, kBigPiece, sK + (buf ^ 1) * kSmallTile, kSmallPiece,
                         kIdSS);
@@ -771,32 +805,20 @@ dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
                         kIdSS);
                 mma_commit(&bars->bar_a);
             }
-        }
-        const bool got2 = mbar_wait_warp(&bars->bar_b, j & 1, &never, budget_ns);
-        if (got2) {
-            tc_fence_after();
-            add_tmem32(tl + kDqColdQ, acc);
-            // K_j (read by S_j and dS_j K_j) and V_j (read by dP_j) are free:
-            // tile j + 2 goes there, tile j + 3 starts arriving.
-            if (j + 2 < T) {
-                split_staged<kSmall, kBwdThreads>(stK, smem + kDqOffK + buf * kSmallTile, tid);
-                split_staged<kSmall, kBwdThreads>(stV, smem + kDqOffV + buf * kSmallTile, tid);
-                fence_proxy_async_smem();
-                if (j + 3 < T) fetch_kv(j + 3);
-            }
-        }
-        tc_fence_before();
-        if (__syncthreads_or(!got2)) {
-            ok = false;
-            break;
+            mma6_ts(tmem + kDqColdQ, tmem + kDqColdS, sK + buf * kSmallTile, kIdTS, false);
+            mma_commit(&bars->bar_b);
         }
     }
 
     if (ok) {
-        if (row < n) store_half(dQ + (size_t(bh) * n + row) * d, 32 * half, acc, d);
-    } else if (tid == 0) {
-        record_device_error(kErrTimeout);
+        ok = mbar_wait_warp(&bars->bar_b, (T - 1) & 1, &never, budget_ns);
+        if (ok) {
+            tc_fence_after();
+            add_tmem32(tl + kDqColdQ, acc);
+            if (row < n) store_half(dQ + (size_t(bh) * n + row) * d, 32 * half, acc, d);
+        }
     }
+    if (!ok && tid == 0) record_device_error(kErrTimeout);
     teardown(bars, tmem, kDqTmemCols, budget_ns);
 }
 
