@@ -124,6 +124,53 @@ __device__ __forceinline__ void load_split(const float* __restrict__ src, int ro
     }
 }
 
+// load_split of two matrices with the same rows (K and V, or Q and dO): all
+// of a thread's loads are issued before any is split, so that the prologue
+// of a CTA waits for memory once rather than once per matrix and chunk.
+template <int R, int NT>
+__device__ __forceinline__ void load_split2(const float* __restrict__ srcA, int widthA, uint8_t* dstA,
+                                            const float* __restrict__ srcB, int widthB, uint8_t* dstB,
+                                            int row0, int rows_valid, int tid) {
+    static_assert((R * 8) % NT == 0, "whole chunks per thread");
+    constexpr int kIters = R * 8 / NT;
+    float4 a[2][kIters], b[2][kIters];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const float* src = m ? srcB : srcA;
+        const int width = m ? widthB : widthA;
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            const int k = tid + it * NT;
+            const int r = k >> 3, col = 8 * (k & 7);
+            const int grow = row0 + r;
+            a[m][it] = b[m][it] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (grow < rows_valid && col < width) {
+                const float4* ptr = reinterpret_cast<const float4*>(src + size_t(grow) * width + col);
+                a[m][it] = __ldg(ptr);
+                if (col + 8 <= width) b[m][it] = __ldg(ptr + 1);
+            }
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        uint8_t* dst = m ? dstB : dstA;
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            const int k = tid + it * NT;
+            const int r = k >> 3, c = k & 7;
+            uint4 p0, p1, p2;
+            split2(a[m][it].x, a[m][it].y, p0.x, p1.x, p2.x);
+            split2(a[m][it].z, a[m][it].w, p0.y, p1.y, p2.y);
+            split2(b[m][it].x, b[m][it].y, p0.z, p1.z, p2.z);
+            split2(b[m][it].z, b[m][it].w, p0.w, p1.w, p2.w);
+            const int off = r * 128 + ((c ^ (r & 7)) << 4);
+            *reinterpret_cast<uint4*>(dst + off) = p0;
+            *reinterpret_cast<uint4*>(dst + R * 128 + off) = p1;
+            *reinterpret_cast<uint4*>(dst + 2 * R * 128 + off) = p2;
+        }
+    }
+}
+
 // Asynchronous 16-byte global -> shared copies (zero-filled past src_bytes).
 __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(sdst)),
@@ -315,11 +362,10 @@ fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K, const float
         // Key tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
         if (T > 2) fetch_kv(2);
         load_split<kBig, kFwdThreads>(Qh, q0, n, d, smem + kFwdOffQ, tid);
-        load_split<kSmall, kFwdThreads>(Kh, 0, m, d, smem + kFwdOffK, tid);
-        load_split<kSmall, kFwdThreads>(Vh, 0, m, dv, smem + kFwdOffV, tid);
+        load_split2<kSmall, kFwdThreads>(Kh, d, smem + kFwdOffK, Vh, dv, smem + kFwdOffV, 0, m, tid);
         if (T > 1) {
-            load_split<kSmall, kFwdThreads>(Kh, kSmall, m, d, smem + kFwdOffK + kSmallTile, tid);
-            load_split<kSmall, kFwdThreads>(Vh, kSmall, m, dv, smem + kFwdOffV + kSmallTile, tid);
+            load_split2<kSmall, kFwdThreads>(Kh, d, smem + kFwdOffK + kSmallTile, Vh, dv,
+                                             smem + kFwdOffV + kSmallTile, kSmall, m, tid);
         }
     }
     fence_proxy_async_smem();
@@ -529,8 +575,8 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
     // rows < n_pad: 64-row tiles never pass the 128-row padding
     auto load_q = [&](int idx, int buf) {
         const int r0 = (i0 + idx) * kSmall;
-        load_split<kSmall, kBwdThreads>(Qh, r0, n, d, smem + kKvOffQ + buf * kSmallTile, tid);
-        load_split<kSmall, kBwdThreads>(dOh, r0, n, dv, smem + kKvOffdO + buf * kSmallTile, tid);
+        load_split2<kSmall, kBwdThreads>(Qh, d, smem + kKvOffQ + buf * kSmallTile, dOh, dv,
+                                         smem + kKvOffdO + buf * kSmallTile, r0, n, tid);
         if (tid < kSmall) sRow[buf * 128 + tid] = L2h[r0 + tid];
         else if (tid < 2 * kSmall) sRow[buf * 128 + tid] = Dh[r0 + tid - kSmall];
     };
@@ -558,8 +604,7 @@ kv_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
     if (aligned) {
         // Query tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
         if (T > 2) fetch_q(2);
-        load_split<kBig, kBwdThreads>(Kh, k0, m, d, smem + kKvOffK, tid);
-        load_split<kBig, kBwdThreads>(Vh, k0, m, dv, smem + kKvOffV, tid);
+        load_split2<kBig, kBwdThreads>(Kh, d, smem + kKvOffK, Vh, dv, smem + kKvOffV, k0, m, tid);
         load_q(0, 0);
         if (T > 1) load_q(1, 1);
     }
@@ -719,13 +764,11 @@ dq_pass(int cta, const float* __restrict__ Q, const float* __restrict__ K, const
     if (aligned) {
         // Key tiles 0 and 1 are split in place; tile 2 is in flight meanwhile.
         if (T > 2) fetch_kv(2);
-        load_split<kBig, kBwdThreads>(Qh, q0, n, d, smem + kDqOffQ, tid);
-        load_split<kBig, kBwdThreads>(dOh, q0, n, dv, smem + kDqOffdO, tid);
-        load_split<kSmall, kBwdThreads>(Kh, 0, m, d, smem + kDqOffK, tid);
-        load_split<kSmall, kBwdThreads>(Vh, 0, m, dv, smem + kDqOffV, tid);
+        load_split2<kBig, kBwdThreads>(Qh, d, smem + kDqOffQ, dOh, dv, smem + kDqOffdO, q0, n, tid);
+        load_split2<kSmall, kBwdThreads>(Kh, d, smem + kDqOffK, Vh, dv, smem + kDqOffV, 0, m, tid);
         if (T > 1) {
-            load_split<kSmall, kBwdThreads>(Kh, kSmall, m, d, smem + kDqOffK + kSmallTile, tid);
-            load_split<kSmall, kBwdThreads>(Vh, kSmall, m, dv, smem + kDqOffV + kSmallTile, tid);
+            load_split2<kSmall, kBwdThreads>(Kh, d, smem + kDqOffK + kSmallTile, Vh, dv,
+                                             smem + kDqOffV + kSmallTile, kSmall, m, tid);
         }
     }
     fence_proxy_async_smem();
