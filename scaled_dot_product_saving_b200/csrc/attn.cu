@@ -363,9 +363,10 @@ attn_status_t bwd_tensor(const void* Q, const void* K, const void* V, const void
     const int grid = static_cast<int>(std::min<long long>(items, sm_count()));
     const int head_group = std::max(1, std::min(BH, 256 / num_kt));
     // A programmatic dependent of the preprocess kernel launched just before
-    // it on the stream: its CTAs set up while the preprocess kernel finishes,
-    // and wait for its results in the kernel (griddepcontrol). Not while
-    // tracing: the early start would then be counted in this kernel's time.
+    // it on the stream: launched early, it waits for that kernel's results in
+    // the kernel (griddepcontrol); its CTAs need an SM's whole register file,
+    // so they start as the preprocess CTAs leave. Not while tracing: the early
+    // start would then be counted in this kernel's time.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(attn::bwdtc::kThreads);

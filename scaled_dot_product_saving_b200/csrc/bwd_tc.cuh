@@ -13,10 +13,10 @@
 //   dK_j += dS^T Q_i                  tcgen05, A = dS^T from TMEM, B = Q_i MN-major
 //   dQ_i += dS K_j                    tcgen05, A = dS from shared memory
 //                                     (MN-major), B = K_j (MN-major); a second
-//                                     warpgroup stages the fp32 result through
-//                                     the (by then free) dS tile and hands it to
-//                                     the TMA engine as tiled reduce-adds into
-//                                     the global dQ accumulator.
+//                                     warpgroup stages the fp32 result in shared
+//                                     memory (d = 128: the by then free dS tile)
+//                                     and hands it to the TMA engine as tiled
+//                                     reduce-adds into the global dQ accumulator.
 // dV_j and dK_j stay in TMEM across all query tiles and are written once.
 // Folding `scale` into dS makes dK and dQ come out already scaled.
 //
@@ -35,8 +35,8 @@
 //
 // Two P/dS warpgroups split a tile into four chunks of 32 queries (two chunks
 // each) and signal each chunk as soon as its P^T/dS^T are in TMEM, so the MMA
-// thread issues that chunk's dV/dK k-steps while the chunks after it are
-// computed; with two warps per SM sub-partition each hides the other's
+// thread issues that chunk's dV/dK k-steps (d = 64: a half's two chunks at a
+// time) while the chunks after it are computed; with two warps per SM sub-partition each hides the other's
 // latencies. Each chunk's P^T/dS^T go into the first 16 of its own 32 TMEM
 // columns, so no chunk overwrites data another chunk has yet to read. dS for
 // the dQ MMA is kept in registers and written to shared memory only at the
@@ -55,8 +55,8 @@
 //
 // Warp roles (512 threads): warps 0-3 and 4-7 = the two P/dS warpgroups (TMEM
 // lane = key), warps 8-11 = dQ warpgroup (TMEM lane = query row), warp 12 =
-// TMA producer, warp 13 = TMEM allocator and MMA issuer, warps 14-15 = dQ
-// converters.
+// TMA producer, warp 13 = TMEM allocator and MMA issuer (the whole warp walks
+// the issue loop, one elected lane issues), warps 14-15 = dQ converters.
 //
 // TMEM (512 columns). d = 128: dV [0,128) dK [128,256) S^T [256,384)
 // dP^T [384,512); chunk c's P^T (bf16) goes to [256+32c, 256+32c+16) and its
@@ -414,9 +414,10 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
     tc_fence_after();
     const uint32_t tmem = bars->tmem_base;
     const bool aborted_early = bars->abort != 0;
-    // Launched as a programmatic dependent of the preprocess kernel: the
-    // setup above overlapped its tail; its outputs (LSE_2, D, the zeroed
-    // accumulator and counters) are touched only after this.
+    // Launched as a programmatic dependent of the preprocess kernel (its
+    // CTAs start on an SM once the preprocess CTAs there have left); its
+    // outputs (LSE_2, D, the zeroed accumulator and counters) are touched
+    // only after this.
     grid_dependency_wait();
 
     // dQ conversion, by one warp: slabs of 32 rows in head order (the order in
