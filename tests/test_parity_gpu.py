@@ -88,6 +88,8 @@ def test_cuda_core_path_bf16(d, causal):
     (2, 40, 700, 700, 128, True),      # 240 forward / 480 backward items: several per CTA, ragged
     (4, 50, 300, 1000, 64, False),     # 400 / 1600 items, n != m, both ragged
     (1, 160, 130, 130, 128, True),     # one-key-tile items and one-tile pairs (has no tile B)
+    (1, 160, 130, 130, 64, True),      # the same at d = 64 (items of one and two query tiles)
+    (3, 37, 1000, 1000, 64, True),     # d = 64, 296 key-tile items in several causal head groups
 ])
 @pytest.mark.parametrize("dq_path", DQ_PATHS, ids=DQ_IDS)
 def test_persistent_many_items(B, H, n, m, d, causal, dq_path):
