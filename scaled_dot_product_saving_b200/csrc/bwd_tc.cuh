@@ -43,8 +43,9 @@
 // end of the tile, by when the dQ warpgroup has normally finished staging the
 // previous tile's dQ through that buffer. Items are ordered head-major, so the
 // key tiles of one head run together and share its Q/dO tiles and its slice
-// of the dQ accumulator through L2. An item's dV/dK epilogue is staged in the
-// Q/dO stage of its last tile and overlaps the next item's first loads.
+// of the dQ accumulator through L2. An item's dV/dK epilogue is the dQ
+// warpgroup's: staged in the Q/dO stage of the item's last tile, it overlaps
+// the next item's first loads and P/dS work.
 //
 // Where the pages stand: dV, dP, dS, dQ and dK are "Attention Backward Pass
 // (dQ, dK, dV)", section "Backward", and "Attention backward", Problems 2-6;
@@ -396,8 +397,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
         mbar_init(&bars->ds_smem_full, C::kSplit ? 256 + 128 : 256);
         mbar_init(&bars->ds_smem_free, 128);
         mbar_init(&bars->acc_done, 1);
-        mbar_init(&bars->acc_free, 256);
-        for (int s = 0; s < 4; ++s) mbar_init(&bars->epi_done[s], 256);
+        mbar_init(&bars->acc_free, 128);
+        for (int s = 0; s < 4; ++s) mbar_init(&bars->epi_done[s], 128);
         mbar_init(&bars->mma_drain, 1);
         for (int k = 0; k < 4; ++k) {
             mbar_init(&bars->sched_full[k], 1);
@@ -812,56 +813,8 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 mbar_arrive(&bars->ds_smem_full);
             }
             if (!ok) break;
-            // Epilogue of item j: group 0 writes dV, group 1 writes dK, staged
-            // in the Q / dO halves of the stage that held the item's last tile
-            // (every MMA that read it is complete once acc_done has fired; the
-            // producer reloads it only after epi_done). Each thread reads its
-            // key row out of TMEM 32 columns at a time, converts it to bf16
-            // and stages it in the 128-byte swizzled layout of the output's
-            // tensor map; one lane per warp stores 32 x 64 boxes with the TMA
-            // (rows past m clipped). The accumulators are released for the
-            // next item as soon as they have been read.
-            if (!mbar_wait_warp(&bars->acc_done, j & 1, abort_flag, budget_ns)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            {
-                const int s_last = (g - 1) % C::kStages;
-                const uint32_t col = grp == 0 ? C::kColdV : C::kColdK;
-                uint8_t* stage = smem + (grp == 0 ? C::kOffQ : C::kOffdO) + s_last * C::kTileBytes +
-                                 (warp & 3) * (32 * D * 2);
-#pragma unroll
-                for (int q = 0; q < D / 32; ++q) {
-                    uint32_t rr[32];
-                    tmem_ld32(tl + col + 32 * q, rr);
-                    tmem_ld_wait(rr);
-                    uint8_t* buf = stage + (q >> 1) * 4096;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int kc = 4 * (q & 1) + k;            // 16-byte chunk of the 128-byte row
-                        *reinterpret_cast<uint4*>(buf + lane * 128 + ((kc ^ (lane & 7)) * 16)) = make_uint4(
-                            pack_bf16x2(__uint_as_float(rr[8 * k + 0]), __uint_as_float(rr[8 * k + 1])),
-                            pack_bf16x2(__uint_as_float(rr[8 * k + 2]), __uint_as_float(rr[8 * k + 3])),
-                            pack_bf16x2(__uint_as_float(rr[8 * k + 4]), __uint_as_float(rr[8 * k + 5])),
-                            pack_bf16x2(__uint_as_float(rr[8 * k + 6]), __uint_as_float(rr[8 * k + 7])));
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&bars->acc_free);
-                const CUtensorMap* out_map = grp == 0 ? &tmdV : &tmdK;
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-#pragma unroll
-                    for (int pnl = 0; pnl < C::kPanels; ++pnl)
-                        tma_store_3d(out_map, stage + pnl * 4096, 64 * pnl, it.k0 + 32 * (warp & 3), it.bh);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();
-                }
-                __syncwarp();
-                mbar_arrive(&bars->epi_done[s_last]);
-            }
+            // The item's dV/dK epilogue is the dQ warpgroup's: this group goes
+            // straight on to the next item.
         }
         if (!ok) {
             record_device_error(kErrTimeout);
@@ -946,6 +899,65 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 if (!C::kSplit) mbar_arrive(&bars->ds_smem_free);
             }
             if (!ok) break;
+            // Epilogue of item j: dV and dK, staged in the Q / dO halves of
+            // the stage that held the item's last tile (every MMA that read it
+            // is complete once acc_done has fired; the producer reloads it
+            // only after epi_done). Each thread reads its key row out of TMEM
+            // 32 columns at a time, converts it to bf16 and stages it in the
+            // 128-byte swizzled layout of the output's tensor map; one lane per
+            // warp stores 32 x 64 boxes with the TMA (rows past m clipped).
+            // The accumulators are released for the next item as soon as they
+            // have been read. Done here rather than by the P/dS warpgroups, so
+            // that they start on the next item at once.
+            if (!mbar_wait_warp(&bars->acc_done, j & 1, abort_flag, budget_ns)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            {
+                const int s_last = (g - 1) % C::kStages;
+#pragma unroll
+                for (int which = 0; which < 2; ++which) {             // dV, then dK
+                    const uint32_t col = which == 0 ? C::kColdV : C::kColdK;
+                    uint8_t* st = smem + (which == 0 ? C::kOffQ : C::kOffdO) + s_last * C::kTileBytes +
+                                  wq * (32 * D * 2);
+#pragma unroll
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t rr[32];
+                        tmem_ld32(tl + col + 32 * q, rr);
+                        tmem_ld_wait(rr);
+                        uint8_t* buf = st + (q >> 1) * 4096;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int kc = 4 * (q & 1) + k;        // 16-byte chunk of the 128-byte row
+                            *reinterpret_cast<uint4*>(buf + lane * 128 + ((kc ^ (lane & 7)) * 16)) = make_uint4(
+                                pack_bf16x2(__uint_as_float(rr[8 * k + 0]), __uint_as_float(rr[8 * k + 1])),
+                                pack_bf16x2(__uint_as_float(rr[8 * k + 2]), __uint_as_float(rr[8 * k + 3])),
+                                pack_bf16x2(__uint_as_float(rr[8 * k + 4]), __uint_as_float(rr[8 * k + 5])),
+                                pack_bf16x2(__uint_as_float(rr[8 * k + 6]), __uint_as_float(rr[8 * k + 7])));
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bars->acc_free);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int which = 0; which < 2; ++which) {
+                        uint8_t* st = smem + (which == 0 ? C::kOffQ : C::kOffdO) + s_last * C::kTileBytes +
+                                      wq * (32 * D * 2);
+#pragma unroll
+                        for (int pnl = 0; pnl < C::kPanels; ++pnl)
+                            tma_store_3d(which == 0 ? &tmdV : &tmdK, st + pnl * 4096, 64 * pnl,
+                                         it.k0 + 32 * wq, it.bh);
+                    }
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+                __syncwarp();
+                mbar_arrive(&bars->epi_done[s_last]);
+            }
             // Every partial of this item has been handed to the TMA: once they
             // have landed, count the item for its head (the converter warps
             // wait for that count). The next item's first dQ is microseconds
