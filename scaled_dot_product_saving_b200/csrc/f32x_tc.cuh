@@ -8,12 +8,12 @@
 // Step by step derivation", section "Gradient of S"): dV = P^T dO,
 // dS = P * (dO V^T - D), dQ = scale dS K, dK = scale dS^T Q.
 //
-// Precision. A value x in fp32 is written as x0 + x1 + x2 with
-//   x0 = bf16(x),  x1 = bf16(x - x0),  x2 = bf16(x - x0 - x1)
-// (both subtractions are exact in fp32), which leaves |x - x0 - x1 - x2| at
-// most about 2^-26 |x|. A product a b is the sum of the six piece products
-// a_i b_j with i + j <= 2; the three left out are below about 2^-25 |a b|
-// together. Each piece product is one bf16 tcgen05 MMA accumulating in fp32
+// Precision. A value x in fp32 is written exactly as x0 + x1 + x2 with
+//   x0 = bf16(x) (rounded to nearest),  x1 = x - x0 truncated to bf16,
+//   x2 = x - x0 - x1 (at most 8 significant bits, so a bf16 value)
+// (both subtractions are exact in fp32); |x1| <= 2^-8 |x| and |x2| < 2^-16
+// |x|. A product a b is the sum of the six piece products a_i b_j with
+// i + j <= 2; the three left out are below about 2^-23 |a b| together. Each piece product is one bf16 tcgen05 MMA accumulating in fp32
 // in TMEM, so one fp32 contraction costs six bf16 MMAs -- the tensor time of
 // three tf32 MMAs (tf32 runs at half the bf16 rate), with operands rounded to
 // 24 significant bits instead of the 22 of a tf32 hi/lo pair, and with the
@@ -82,17 +82,19 @@ __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) {
 }
 
 // Two fp32 values (x: lower element) into their three bf16 pieces, packed
-// two to a word.
+// two to a word: x0 = bf16(x) rounded to nearest, x1 = x - x0 truncated to
+// bf16 (its upper 16 bits), x2 = x - x0 - x1. Both subtractions are exact,
+// and x2 has at most 8 significant bits, so x0 + x1 + x2 = x exactly with one
+// float-to-bf16 conversion per pair (the conversion pipe is the narrow one).
 __device__ __forceinline__ void split2(float x, float y, uint32_t& w0, uint32_t& w1, uint32_t& w2) {
     const __nv_bfloat162 h0 = __floats2bfloat162_rn(x, y);
     const float2 f0 = __bfloat1622float2(h0);
     const float rx = __fsub_rn(x, f0.x), ry = __fsub_rn(y, f0.y);
-    const __nv_bfloat162 h1 = __floats2bfloat162_rn(rx, ry);
-    const float2 f1 = __bfloat1622float2(h1);
-    const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fsub_rn(rx, f1.x), __fsub_rn(ry, f1.y));
+    const uint32_t ux = __float_as_uint(rx) & 0xffff0000u, uy = __float_as_uint(ry) & 0xffff0000u;
+    const float sx = __fsub_rn(rx, __uint_as_float(ux)), sy = __fsub_rn(ry, __uint_as_float(uy));
     w0 = bf2_bits(h0);
-    w1 = bf2_bits(h1);
-    w2 = bf2_bits(h2);
+    w1 = __byte_perm(ux, uy, 0x7632);
+    w2 = __byte_perm(__float_as_uint(sx), __float_as_uint(sy), 0x7632);
 }
 
 // Rows [row0, row0 + R) of a row-major [rows_valid, width] fp32 matrix into
