@@ -571,12 +571,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             const int s = g % C::kStages;
             if (!mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns)) return false;
             tc_fence_after();
-            const uint32_t sdO = smem_addr(smem + C::kOffdO + s * C::kTileBytes);
+            const uint64_t aV = sdesc_sw128(sV, 16, 1024);
+            const uint64_t bdO = sdesc_sw128(smem_addr(smem + C::kOffdO + s * C::kTileBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::col_dp(0), sdesc_sw128(sV + koff, 16, 1024),
-                         sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0, leader);
+                mma_ss_w(tmem + C::col_dp(0), sdesc_adv(aV, koff), sdesc_adv(bdO, koff), idSP, kk > 0,
+                         leader);
             }
             return true;
         };
@@ -588,12 +589,13 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 !mbar_wait_warp(&bars->dq_free, (g - 1) & 1, abort_flag, budget_ns))
                 return false;
             tc_fence_after();
-            const uint32_t sQ = smem_addr(smem + C::kOffQ + (g % C::kStages) * C::kTileBytes);
+            const uint64_t aK = sdesc_sw128(sK, 16, 1024);
+            const uint64_t bQ =
+                sdesc_sw128(smem_addr(smem + C::kOffQ + (g % C::kStages) * C::kTileBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::col_s(0), sdesc_sw128(sK + koff, 16, 1024),
-                         sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0, leader);
+                mma_ss_w(tmem + C::col_s(0), sdesc_adv(aK, koff), sdesc_adv(bQ, koff), idSP, kk > 0, leader);
             }
             mma_commit_w(&bars->s_full[0], leader);
             return true;
@@ -608,19 +610,20 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             if (h == 0 && !mbar_wait_warp(&bars->q_full[s], (g / C::kStages) & 1, abort_flag, budget_ns))
                 return false;
             tc_fence_after();
-            const uint32_t sQh = smem_addr(smem + C::kOffQ + s * C::kTileBytes) + h * 8192;
-            const uint32_t sdOh = smem_addr(smem + C::kOffdO + s * C::kTileBytes) + h * 8192;
+            const uint64_t bQh = sdesc_sw128(smem_addr(smem + C::kOffQ + s * C::kTileBytes) + h * 8192, 16, 1024);
+            const uint64_t bdOh = sdesc_sw128(smem_addr(smem + C::kOffdO + s * C::kTileBytes) + h * 8192, 16, 1024);
+            const uint64_t aV = sdesc_sw128(sV, 16, 1024), aK = sdesc_sw128(sK, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::col_dp(2 * h), sdesc_sw128(sV + koff, 16, 1024),
-                         sdesc_sw128(sdOh + koff, 16, 1024), idHalf, kk > 0, leader);
+                mma_ss_w(tmem + C::col_dp(2 * h), sdesc_adv(aV, koff), sdesc_adv(bdOh, koff), idHalf, kk > 0,
+                         leader);
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::col_s(2 * h), sdesc_sw128(sK + koff, 16, 1024),
-                         sdesc_sw128(sQh + koff, 16, 1024), idHalf, kk > 0, leader);
+                mma_ss_w(tmem + C::col_s(2 * h), sdesc_adv(aK, koff), sdesc_adv(bQh, koff), idHalf, kk > 0,
+                         leader);
             }
             mma_commit_w(&bars->s_full[h], leader);
             return true;
@@ -664,14 +667,16 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                 // and 3. d = 64: a half at a time (its warpgroup signals chunk
                 // 2h+1 after chunk 2h), then the half's next S^T/dP^T.
                 bool first = (t == 0);
+                const uint64_t bdO = sdesc_sw128(sdO, C::kPanelBytes, 1024);
+                const uint64_t bQ = sdesc_sw128(sQ, C::kPanelBytes, 1024);
                 auto issue_chunk = [&](int c) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
-                        mma_ts_w(tmem + C::kColdV, tmem + C::col_s(c) + 8 * h,
-                                 sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
-                        mma_ts_w(tmem + C::kColdK, tmem + C::col_dp(c) + 8 * h,
-                                 sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
+                        mma_ts_w(tmem + C::kColdV, tmem + C::col_s(c) + 8 * h, sdesc_adv(bdO, kk * 2048), idKV,
+                                 !first, leader);
+                        mma_ts_w(tmem + C::kColdK, tmem + C::col_dp(c) + 8 * h, sdesc_adv(bQ, kk * 2048), idKV,
+                                 !first, leader);
                         first = false;
                     }
                 };
@@ -709,10 +714,12 @@ bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
                     break;
                 }
                 tc_fence_after();
+                const uint64_t aS = sdesc_sw128(sdS, C::kPanelBytes, 1024);
+                const uint64_t bK = sdesc_sw128(sK, C::kPanelBytes, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ss_w(tmem + C::kColdQ, sdesc_sw128(sdS + kk * 2048, C::kPanelBytes, 1024),
-                             sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, kk > 0, leader);
+                    mma_ss_w(tmem + C::kColdQ, sdesc_adv(aS, kk * 2048), sdesc_adv(bK, kk * 2048), idQ, kk > 0,
+                             leader);
                 mma_commit_w(&bars->dq_full, leader);
                 // The item's last MMA has been issued: K_j, V_j are free once
                 // it has completed.

@@ -382,7 +382,7 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 // K-major: rows of 128 B (64 bf16 along K), 8-row groups `sbo` bytes apart.
 // MN-major: 64 bf16 along M/N per 128 B row, K rows 128 B apart, 8-row K
 // groups `sbo` apart, and 64-wide M/N panels `lbo` bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+__host__ __device__ constexpr uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
     d |= uint64_t((saddr >> 4) & 0x3FFFu);
     d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
@@ -391,6 +391,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
     d |= uint64_t(2) << 61;
     return d;
 }
+
+// The descriptor of the same operand `bytes` further on (a multiple of 16).
+// Shared-memory addresses stay below 256 KB, so the start field never carries
+// into the bits above it: one 32-bit add on the low word instead of building
+// the descriptor again for every k-step.
+__host__ __device__ constexpr uint64_t sdesc_adv(uint64_t d, uint32_t bytes) {
+    return (uint64_t(uint32_t(d >> 32)) << 32) | uint32_t(uint32_t(d) + (bytes >> 4));
+}
+static_assert(sdesc_adv(sdesc_sw128(0x1400, 16, 1024), 0x7e0) == sdesc_sw128(0x1be0, 16, 1024),
+              "advanced descriptor");
+static_assert(sdesc_adv(sdesc_sw128(0x30000, 8192, 1024), 0x8ff0) == sdesc_sw128(0x38ff0, 8192, 1024),
+              "advanced descriptor near the top of shared memory");
 
 // TMEM -> registers: 32 lanes x 32 bit, 32 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
