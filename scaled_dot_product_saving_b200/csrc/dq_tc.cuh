@@ -309,8 +309,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColS0 + 128 * (c & 1), sdesc_sw128(sQ + koff, 16, 1024),
-                         sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0, leader);
+                mma_ss_w(tmem + C::kColS0 + 128 * (c & 1), sdesc_at(sQ, koff, 16, 1024),
+                         sdesc_at(sK, koff, 16, 1024), idS, kk > 0, leader);
             }
             mma_commit_w(&bars->s_full[c & 1], leader);
         };
@@ -319,8 +319,8 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sdO + koff, 16, 1024),
-                         sdesc_sw128(sV + koff, 16, 1024), idS, kk > 0, leader);
+                mma_ss_w(tmem + C::kColdP, sdesc_at(sdO, koff, 16, 1024),
+                         sdesc_at(sV, koff, 16, 1024), idS, kk > 0, leader);
             }
             mma_commit_w(&bars->dp_full, leader);
         };
@@ -376,7 +376,7 @@ dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)          // keys 16kk .. 16kk+15
                     mma_ts_w(tmem + C::kColdQ, sbuf + 64 * (kk >> 2) + 8 * (kk & 3),
-                             sdesc_sw128(sK + kk * 2048, C::kPanelBytes, 1024), idQ, t > 0 || kk > 0, leader);
+                             sdesc_at(sK, kk * 2048, C::kPanelBytes, 1024), idQ, t > 0 || kk > 0, leader);
                 mma_commit_w(&bars->k_empty[g % C::kKStages], leader);
                 if (t == it.nkv - 1) mma_commit_w(&bars->dq_done, leader);
             }

@@ -249,8 +249,8 @@ __device__ __forceinline__ void mma6_ss(uint32_t d, uint32_t sa, uint32_t a_stri
     for (int p = 0; p < 6; ++p)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_ss(d, sdesc_sw128(sa + pair_a(p) * a_stride + kk * 32, 16, 1024),
-                   sdesc_sw128(sb + pair_b(p) * b_stride + kk * 32, 16, 1024), idesc,
+            mma_ss(d, sdesc_at(sa + pair_a(p) * a_stride, kk * 32, 16, 1024),
+                   sdesc_at(sb + pair_b(p) * b_stride, kk * 32, 16, 1024), idesc,
                    (p > 0 || kk > 0) ? 1u : 0u);
 }
 
@@ -264,7 +264,7 @@ __device__ __forceinline__ void mma6_ts(uint32_t d, uint32_t ta, uint32_t sb, ui
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
             mma_ts(d, ta + 32 * pair_a(p) + 8 * kk,
-                   sdesc_sw128(sb + pair_b(p) * kSmallPiece + kk * 2048, kSmallPiece, 1024), idesc,
+                   sdesc_at(sb + pair_b(p) * kSmallPiece, kk * 2048, kSmallPiece, 1024), idesc,
                    (accumulate || p > 0 || kk > 0) ? 1u : 0u);
 }
 

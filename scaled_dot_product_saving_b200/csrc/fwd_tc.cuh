@@ -357,8 +357,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColS0 + 128 * x, sdesc_sw128(sQ + koff, 16, 1024),
-                         sdesc_sw128(sK + koff, 16, 1024), idS, kk > 0, leader);
+                mma_ss_w(tmem + C::kColS0 + 128 * x, sdesc_at(sQ, koff, 16, 1024),
+                         sdesc_at(sK, koff, 16, 1024), idS, kk > 0, leader);
             }
             mma_commit_w(&bars->s_full[x], leader);
         };
@@ -370,7 +370,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUte
             for (int k4 = 0; k4 < 4; ++k4) {
                 const int kk = 4 * h + k4;
                 mma_ts_w(tmem + C::kColO0 + D * x, tmem + C::kColS0 + 128 * x + kk * 8,
-                         sdesc_sw128(sV + kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0), leader);
+                         sdesc_at(sV, kk * 2048, C::kPanelBytes, 1024), idO, (t > 0 || kk > 0), leader);
             }
         };
         bool ok = true;

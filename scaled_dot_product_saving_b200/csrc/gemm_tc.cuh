@@ -138,10 +138,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
             for (int kk = 0; kk < kBK / 16; ++kk) {
                 // K-major: a K step is 32 bytes along the 128-byte row;
                 // MN-major: 16 rows of 128 bytes, 64-wide panels 8 KB apart.
-                const uint64_t da = A_KMAJOR ? sdesc_sw128(sa + kk * 32, 16, 1024)
-                                             : sdesc_sw128(sa + kk * 2048, 8192, 1024);
-                const uint64_t db = B_KMAJOR ? sdesc_sw128(sb + kk * 32, 16, 1024)
-                                             : sdesc_sw128(sb + kk * 2048, 8192, 1024);
+                const uint64_t da = A_KMAJOR ? sdesc_at(sa, kk * 32, 16, 1024)
+                                             : sdesc_at(sa, kk * 2048, 8192, 1024);
+                const uint64_t db = B_KMAJOR ? sdesc_at(sb, kk * 32, 16, 1024)
+                                             : sdesc_at(sb, kk * 2048, 8192, 1024);
                 mma_ss_w(tmem, da, db, idesc, (kb > 0 || kk > 0) ? 1u : 0u, leader);
             }
             mma_commit_w(&bars->empty[s], leader);

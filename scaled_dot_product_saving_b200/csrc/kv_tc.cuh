@@ -383,8 +383,8 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColS, sdesc_sw128(sK + koff, 16, 1024),
-                         sdesc_sw128(sQ + koff, 16, 1024), idSP, kk > 0, leader);
+                mma_ss_w(tmem + C::kColS, sdesc_at(sK, koff, 16, 1024),
+                         sdesc_at(sQ, koff, 16, 1024), idSP, kk > 0, leader);
             }
             mma_commit_w(&bars->s_full, leader);
             return true;
@@ -394,8 +394,8 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t koff = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-                mma_ss_w(tmem + C::kColdP, sdesc_sw128(sV + koff, 16, 1024),
-                         sdesc_sw128(sdO + koff, 16, 1024), idSP, kk > 0, leader);
+                mma_ss_w(tmem + C::kColdP, sdesc_at(sV, koff, 16, 1024),
+                         sdesc_at(sdO, koff, 16, 1024), idSP, kk > 0, leader);
             }
             mma_commit_w(&bars->dp_full, leader);
         };
@@ -437,7 +437,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;                      // queries 16kk..16kk+15
                         mma_ts_w(tmem + C::kColdV, tmem + C::kColP + 32 * c + 8 * h,
-                                 sdesc_sw128(sdO + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
+                                 sdesc_at(sdO, kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
                 }
@@ -457,7 +457,7 @@ kv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUten
                     for (int h = 0; h < 2; ++h) {
                         const int kk = 2 * c + h;
                         mma_ts_w(tmem + C::kColdK, tmem + C::kColdS + 32 * c + 8 * h,
-                                 sdesc_sw128(sQ + kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
+                                 sdesc_at(sQ, kk * 2048, C::kPanelBytes, 1024), idKV, !first, leader);
                         first = false;
                     }
                 }

@@ -399,6 +399,11 @@ __host__ __device__ constexpr uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo,
 __host__ __device__ constexpr uint64_t sdesc_adv(uint64_t d, uint32_t bytes) {
     return (uint64_t(uint32_t(d >> 32)) << 32) | uint32_t(uint32_t(d) + (bytes >> 4));
 }
+// The descriptor of `base + bytes`, written so that the part that depends on
+// `base` alone is shared by all the k-steps of an unrolled loop.
+__host__ __device__ constexpr uint64_t sdesc_at(uint32_t base, uint32_t bytes, uint32_t lbo, uint32_t sbo) {
+    return sdesc_adv(sdesc_sw128(base, lbo, sbo), bytes);
+}
 static_assert(sdesc_adv(sdesc_sw128(0x1400, 16, 1024), 0x7e0) == sdesc_sw128(0x1be0, 16, 1024),
               "advanced descriptor");
 static_assert(sdesc_adv(sdesc_sw128(0x30000, 8192, 1024), 0x8ff0) == sdesc_sw128(0x38ff0, 8192, 1024),
