@@ -41,9 +41,10 @@
 // columns, so no chunk overwrites data another chunk has yet to read. dS for
 // the dQ MMA is kept in registers and written to shared memory only at the
 // end of the tile, by when the dQ warpgroup has normally finished staging the
-// previous tile's dQ through that buffer. Items are ordered head-major, so the
-// key tiles of one head run together and share its Q/dO tiles and its slice
-// of the dQ accumulator through L2. An item's dV/dK epilogue is the dQ
+// previous tile's dQ through that buffer. Items are ordered in groups of
+// heads, key-tile major inside a group (the longest items first when causal),
+// so the heads in flight share their Q/dO tiles and their slices of the dQ
+// accumulator through L2. An item's dV/dK epilogue is the dQ
 // warpgroup's: staged in the Q/dO stage of the item's last tile, it overlaps
 // the next item's first loads and P/dS work.
 //

@@ -30,10 +30,11 @@
 // S^T(g+1) (every MMA that reads P^T(g) is issued by then, and the tensor
 // pipe runs MMAs in issue order), then dK(g) chunk by chunk, then dP^T(g+1)
 // (likewise after the last reader of dS^T(g)). So the next tile's phase A
-// overlaps this tile's dK and dP^T MMAs. Items are ordered head-major in
-// groups, longest first, so the key tiles of one head run together and share
-// its Q/dO tiles through L2. An item's dV/dK epilogue is staged in the Q/dO
-// stage of its last tile and overlaps the next item's first loads.
+// overlaps this tile's dK and dP^T MMAs. Items are ordered in groups of
+// heads, key-tile major inside a group (the longest items first when causal),
+// so the heads in flight share their Q/dO tiles through L2. An item's dV/dK
+// epilogue is staged in the Q/dO stage of its last tile and overlaps the next
+// item's first loads.
 //
 // Where the pages stand: dV, dP, dS and dK are "Attention Backward Pass (dQ,
 // dK, dV)", section "Backward", and "Attention backward", Problems 2-6;
