@@ -238,3 +238,18 @@ def test_kernel_names_match_the_header(L):
     body = body[:body.index("attn_kernel_id_t")]
     ids = {int(v) for v in re.findall(r"ATTN_KERNEL_[A-Z0-9_]+\s*=\s*(\d+)", body)}
     assert ids == set(L.KERNEL_NAMES), (ids, sorted(L.KERNEL_NAMES))
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    """No CPU fallback: the binding refuses to import when libattn.so is
+    absent, rather than running anything in Python."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "scaled_dot_product_saving_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "scaled_dot_product_saving_b200", "__init__.py"), pkg)
+    r = subprocess.run([sys.executable, "-c", "import scaled_dot_product_saving_b200"],
+                       cwd=tmp_path, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "libattn.so is missing" in r.stderr
