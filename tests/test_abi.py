@@ -63,6 +63,8 @@ def test_argument_checks_forward(L):
     assert fwd(L, n=0) == 2
     assert fwd(L, n=64, m=65, causal=1) == 2          # causal needs n == m
     assert fwd(L, n=1 << 24, m=1 << 24) == 2
+    assert fwd(L, n=64, m=1 << 24) == 2
+    assert fwd(L, B=1 << 16, H=1 << 15) == 2          # B*H must stay below 2^31
     assert fwd(L, dt=7) == 3
     assert fwd(L, d=129) == 4
     assert fwd(L, q=MIS) == 5
